@@ -1,0 +1,482 @@
+"""Benchmark of the exact-attention hot path on B200.
+
+One step = one pass of the whole path: the tiled forward on the GQA causal long-context
+workload (B=1, Hq=64, Hkv=8, N=8192, d=128, bf16) and the split-KV decode on the decode
+workload (B=8, Hq=64, Hkv=8, cache 32768, d=128, splits of 1024).  The headline value is the
+forward's TFLOP/s (4 B Hq N^2 d, halved for causal); the decode's HBM GB/s (K and V bytes
+read once) is reported in the "decode" object.  Inputs are synthetic i.i.d. N(0,1) from the
+seeded generator, resident in HBM before timing; L2 is flushed (a 256 MiB write) before every
+timed launch, outside its events.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
+
+With N > 1 (launched by torch.distributed.run) every rank runs its own replica of the
+workload (the units are independent: no collective on the data path); times are the max
+over ranks.  --impl reference times the fp64 CPU oracle on bounded samples of the same
+workloads instead.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+
+import synth_inputs as si  # noqa: E402
+
+METRIC = "attention fwd TFLOP/s & % of BF16 tensor peak; decode HBM GB/s & % of peak"
+SPEC_BF16_TFLOPS = 2250.0
+SPEC_HBM_GBS = 8000.0
+FALLBACK_HBM_GBS = 6650.0
+FALLBACK_BF16_TFLOPS = 1590.0
+
+FWD = si.WORKLOADS["gqa_causal_8k"]
+DEC = si.WORKLOADS["decode_split_kv"]
+
+
+def fwd_flops(w=FWD) -> float:
+    f = 4.0 * w["B"] * w["Hq"] * w["N"] * w["N"] * w["d"]
+    return f / 2 if w["causal"] else f
+
+
+def fwd_bytes(w=FWD) -> float:
+    B, N, Hq, Hkv, d = w["B"], w["N"], w["Hq"], w["Hkv"], w["d"]
+    return 2.0 * B * N * Hq * d * 2 + 2.0 * 2 * B * N * Hkv * d + 4.0 * B * Hq * N
+
+
+def dec_kv_bytes(w=DEC) -> float:
+    return 2.0 * w["B"] * w["L"] * w["Hkv"] * w["d"] * 2
+
+
+def dec_flops(w=DEC) -> float:
+    return 4.0 * w["B"] * w["Hq"] * w["L"] * w["d"]
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            j = json.load(f)
+        return {"hbm": j["hbm_gbs"], "bf16": j["bf16_tflops"], "bf16_sustained": j["bf16_tflops_sustained"],
+                "source": "measured"}
+    return {"hbm": FALLBACK_HBM_GBS, "bf16": FALLBACK_BF16_TFLOPS, "bf16_sustained": 1400.0, "source": "fallback"}
+
+
+def kernel_src_hash() -> str:
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "exact_io_aware_97_b200", "csrc")
+    for f in sorted(os.listdir(csrc)):
+        with open(os.path.join(csrc, f), "rb") as fh:
+            h.update(f.encode() + fh.read())
+    return h.hexdigest()[:16]
+
+
+def ncu_traffic(key: str):
+    """DRAM bytes per launch from a committed ncu summary, if taken on the current kernels."""
+    p = os.path.join(ROOT, "profiles", "ncu_traffic.json")
+    if not os.path.exists(p):
+        return None
+    with open(p) as f:
+        j = json.load(f)
+    e = j.get(key)
+    if not e or e.get("src_sha") != kernel_src_hash():
+        return None
+    return e.get("bytes_per_launch")
+
+
+# ----------------------------------------------------------------------------- clocks
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.lines = []
+        self.marks = []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                                          "-lms", "100", "-i", str(self.gpu)], stdout=subprocess.PIPE,
+                                         stderr=subprocess.DEVNULL, text=True)
+            self.t = threading.Thread(target=self._read, daemon=True)
+            self.t.start()
+        except (OSError, ValueError):
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append((time.time(), line.strip()))
+
+    def mark(self, on: bool):
+        self.marks.append((time.time(), on))
+
+    def stop(self):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        if not self.lines:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        # samples inside timed windows
+        wins, cur = [], None
+        for t, on in self.marks:
+            if on:
+                cur = t
+            elif cur is not None:
+                wins.append((cur, t))
+                cur = None
+        inside = [l for t, l in self.lines if any(a - 0.15 <= t <= b + 0.15 for a, b in wins)] or [l for _, l in self.lines]
+        sm, smax, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for l in inside:
+            parts = [x.strip() for x in l.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                smax = float(parts[2])
+            except ValueError:
+                continue
+            for n, val in zip(names, parts[5:9]):
+                if val.lower().startswith("active"):
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": smax, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ----------------------------------------------------------------------------- device arm
+def run_device(args):
+    import torch
+    import torch.distributed as dist
+
+    from exact_io_aware_97_b200 import binding as fa
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    fa.load()
+    peaks = load_peaks()
+    st = torch.cuda.current_stream()
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+
+    def max_over_ranks(x: float) -> float:
+        if world == 1:
+            return x
+        t = torch.tensor([x], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+
+    def l2_flush():
+        flush.fill_(1)
+
+    # ---- inputs (each rank its own replica, seeded by the workload seed + rank)
+    w = FWD
+    B, N, Hq, Hkv, d = w["B"], w["N"], w["Hq"], w["Hkv"], w["d"]
+    seed = w["seed"] + 100000 * rank
+    h_q = torch.from_numpy(si.normal(seed, si.Q, (B, N, Hq, d))).to(torch.bfloat16).pin_memory()
+    h_k = torch.from_numpy(si.normal(seed, si.K, (B, N, Hkv, d))).to(torch.bfloat16).pin_memory()
+    h_v = torch.from_numpy(si.normal(seed, si.V, (B, N, Hkv, d))).to(torch.bfloat16).pin_memory()
+    q, k, v = h_q.to(dev), h_k.to(dev), h_v.to(dev)
+    o = torch.empty_like(q)
+    lse = torch.empty((B, Hq, N), dtype=torch.float32, device=dev)
+    h_o = torch.empty(o.shape, dtype=torch.bfloat16).pin_memory()
+    h_lse = torch.empty(lse.shape, dtype=torch.float32).pin_memory()
+    scale = 1.0 / math.sqrt(d)
+
+    wd = DEC
+    dseed = wd["seed"] + 100000 * rank
+    dB, dHq, dHkv, L, dd, split = wd["B"], wd["Hq"], wd["Hkv"], wd["L"], wd["d"], wd["split"]
+    h_dq = torch.from_numpy(si.normal(dseed, si.Q, (dB, dHq, dd))).to(torch.bfloat16).pin_memory()
+    h_kc = torch.from_numpy(si.normal(dseed, si.KCACHE, (dB, L, dHkv, dd))).to(torch.bfloat16).pin_memory()
+    h_vc = torch.from_numpy(si.normal(dseed, si.VCACHE, (dB, L, dHkv, dd))).to(torch.bfloat16).pin_memory()
+    dq, kc, vc = h_dq.to(dev), h_kc.to(dev), h_vc.to(dev)
+    do = torch.empty((dB, dHq, dd), dtype=torch.bfloat16, device=dev)
+    dlse = torch.empty((dB, dHq), dtype=torch.float32, device=dev)
+    ws_bytes = fa.fa_decode_workspace_size(dB, dHq, L, dd, split)
+    ws = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
+    h_do = torch.empty(do.shape, dtype=torch.bfloat16).pin_memory()
+    dscale = 1.0 / math.sqrt(dd)
+
+    def call_fwd():
+        fa.fa_fwd(q, k, v, o, lse, B, Hq, Hkv, N, N, d, scale, 1, None, fa.FA_BF16, None, 0, st)
+
+    def call_dec(qq=None, kk=None, vv=None):
+        fa.fa_decode(qq if qq is not None else dq, kk if kk is not None else kc, vv if vv is not None else vc, None,
+                     do, dlse, dB, dHq, dHkv, L, dd, dscale, split, ws, ws_bytes, st)
+
+    clocks = ClockSampler(local)
+    clocks.start()
+    time.sleep(0.3)
+
+    def timed_launches(fn, steps, warmup):
+        for _ in range(warmup):
+            l2_flush()
+            fn()
+        barrier()
+        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+        clocks.mark(True)
+        for a, b in evs:
+            l2_flush()
+            a.record(st)
+            fn()
+            b.record(st)
+        barrier()
+        clocks.mark(False)
+        ms = [a.elapsed_time(b) for a, b in evs]
+        return ms
+
+    fwd_ms = timed_launches(call_fwd, args.steps, args.warmup)
+    dec_ms = timed_launches(call_dec, args.steps, args.warmup)
+    if fa.fa_last_device_error(st) != fa.FA_OK:
+        raise RuntimeError("device-side timeout recorded during the benchmark")
+
+    # ---- end to end through the C ABI with host buffers (copies inside the timed region)
+    def e2e(steps, warmup, body):
+        for _ in range(warmup):
+            body()
+        barrier()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        clocks.mark(True)
+        a.record(st)
+        for _ in range(steps):
+            body()
+        b.record(st)
+        barrier()
+        clocks.mark(False)
+        return a.elapsed_time(b) / steps
+
+    def fwd_e2e_body():
+        q.copy_(h_q, non_blocking=True)
+        k.copy_(h_k, non_blocking=True)
+        v.copy_(h_v, non_blocking=True)
+        call_fwd()
+        h_o.copy_(o, non_blocking=True)
+        h_lse.copy_(lse, non_blocking=True)
+
+    def dec_e2e_body():
+        dq.copy_(h_dq, non_blocking=True)
+        kc.copy_(h_kc, non_blocking=True)
+        vc.copy_(h_vc, non_blocking=True)
+        call_dec()
+        h_do.copy_(do, non_blocking=True)
+
+    e2e_steps = max(3, args.steps // 4)
+    fwd_e2e_ms = e2e(e2e_steps, 1, fwd_e2e_body)
+    dec_e2e_ms = e2e(e2e_steps, 1, dec_e2e_body)
+    torch.cuda.synchronize()
+    clocks.stop()
+
+    # ---- reduce over ranks (max time)
+    fwd_mean = max_over_ranks(sum(fwd_ms) / len(fwd_ms))
+    dec_mean = max_over_ranks(sum(dec_ms) / len(dec_ms))
+    fwd_e2e_ms = max_over_ranks(fwd_e2e_ms)
+    dec_e2e_ms = max_over_ranks(dec_e2e_ms)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank != 0:
+        return
+
+    F = fwd_flops()
+    tflops = world * F / (fwd_mean * 1e-3) / 1e12
+    kv = dec_kv_bytes()
+    gbs = world * kv / (dec_mean * 1e-3) / 1e9
+    h2d_fwd = h_q.numel() * 2 + h_k.numel() * 2 + h_v.numel() * 2
+    d2h_fwd = h_o.numel() * 2 + h_lse.numel() * 4
+    h2d_dec = h_dq.numel() * 2 + h_kc.numel() * 2 + h_vc.numel() * 2
+    d2h_dec = h_do.numel() * 2
+    burst = (args.steps * fwd_mean) < 1000.0
+    tc_peak = peaks["bf16"] if burst else peaks["bf16_sustained"]
+    per_launch_tflops = F / (fwd_mean * 1e-3) / 1e12
+    per_launch_gbs = kv / (dec_mean * 1e-3) / 1e9
+    cpu = cpu_baseline_fwd(args.cpu_seconds) if not args.no_cpu else None
+    dec_cpu = cpu_baseline_dec(args.cpu_seconds) if not args.no_cpu else None
+    line = {
+        "metric": METRIC,
+        "value": round(tflops, 2),
+        "unit": "TFLOP/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": round(fwd_mean + dec_mean, 4),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16",
+        "data": "synthetic: i.i.d. N(0,1) from seeded splitmix64 + Box-Muller, rounded to bf16",
+        "config": {"workload": "gqa_causal_8k: B=1, Hq=64, Hkv=8, N=8192, d=128, causal, layout [B,N,H,d]",
+                   "decode_workload": "decode_split_kv: B=8, Hq=64, Hkv=8, cache 32768, d=128, split 1024",
+                   "parallelism": f"replicas x{world} (independent units, no collective)",
+                   "l2": "flushed before every timed launch (256 MiB write, outside the events)",
+                   "timing": "CUDA events around each launch on the launching stream; mean over steps; max over ranks"},
+        "roofline": {"bound": "tensor", "achieved": round(per_launch_tflops, 2), "peak": tc_peak, "unit": "TFLOP/s",
+                     "frac": round(per_launch_tflops / tc_peak, 4),
+                     "peak_kind": ("measured burst" if burst else "measured sustained") + f" ({peaks['source']})",
+                     "frac_of_spec_2250": round(per_launch_tflops / SPEC_BF16_TFLOPS, 4),
+                     "traffic": ncu_traffic("fa_fwd/gqa_causal_8k"),
+                     "kernel": "fa_fwd_kernel<128,false>", "algorithmic_flops_per_launch": F,
+                     "algorithmic_bytes_per_launch": fwd_bytes()},
+        "decode": {"value": round(gbs, 1), "unit": "GB/s", "ms": round(dec_mean, 4),
+                   "roofline": {"bound": "hbm", "achieved": round(per_launch_gbs, 1), "peak": peaks["hbm"],
+                                "unit": "GB/s", "frac": round(per_launch_gbs / peaks["hbm"], 4),
+                                "peak_kind": f"measured copy ({peaks['source']})",
+                                "frac_of_spec_8000": round(per_launch_gbs / SPEC_HBM_GBS, 4),
+                                "traffic": ncu_traffic("fa_decode/decode_split_kv"),
+                                "kernels": "fa_decode_split_kernel<128> + fa_decode_combine_kernel<128>",
+                                "algorithmic_bytes_per_launch": kv,
+                                "tflops": round(dec_flops() / (dec_mean * 1e-3) / 1e12, 2)},
+                   "e2e": {"value": round(world * kv / (dec_e2e_ms * 1e-3) / 1e9, 1), "unit": "GB/s",
+                           "h2d_bytes_per_step": h2d_dec, "d2h_bytes_per_step": d2h_dec},
+                   "cpu_baseline": dec_cpu},
+        "e2e": {"value": round(world * F / (fwd_e2e_ms * 1e-3) / 1e12, 2), "unit": "TFLOP/s",
+                "h2d_bytes_per_step": h2d_fwd, "d2h_bytes_per_step": d2h_fwd},
+        "cpu_baseline": cpu,
+        "gpu_launches": args.steps * 1 + args.steps * 2,
+        "clocks": clocks.summary(),
+        "impl": "b200",
+    }
+    print(json.dumps(line), flush=True)
+
+
+# ----------------------------------------------------------------------------- CPU oracle
+def _oracle_rows_fwd(orc, rows_target, threads, seed):
+    """Time the oracle on `rows_target` random rows of the forward workload."""
+    w = FWD
+    B, N, Hq, Hkv, d = w["B"], w["N"], w["Hq"], w["Hkv"], w["d"]
+    q = si.normal(seed, si.Q, (B, N, Hq, d))
+    k = si.normal(seed, si.K, (B, N, Hkv, d))
+    v = si.normal(seed, si.V, (B, N, Hkv, d))
+    u = si.uniform_ints(seed, 13, 2 * rows_target, 0, (1 << 30))
+    rows = np.stack([np.zeros(rows_target, np.int64), u[0::2] % Hq, u[1::2] % N], 1)
+    t = time.perf_counter()
+    orc.attention_rows(q, k, v, 1.0 / math.sqrt(d), rows, causal=True, nthreads=threads)
+    dt = time.perf_counter() - t
+    flops = float(np.sum(4.0 * (rows[:, 2] + 1) * d))
+    return dt, flops, rows_target
+
+
+def cpu_baseline_fwd(seconds: float):
+    import oracle
+    orc = oracle.get()
+    threads = orc.hardware_threads()
+    dt, fl, n = _oracle_rows_fwd(orc, 256, threads, FWD["seed"])
+    target = max(256, int(n * seconds / max(dt, 1e-3)))
+    dt, fl, n = _oracle_rows_fwd(orc, target, threads, FWD["seed"])
+    return {"value": round(fl / dt / 1e12, 6), "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
+            "sample": f"{n} random causal rows of the gqa_causal_8k workload (fp64, materialised rows), "
+                      f"{dt:.1f} s on {threads} threads"}
+
+
+def _oracle_dec(orc, pairs, threads, seed):
+    w = DEC
+    B, Hq, Hkv, L, d = w["B"], w["Hq"], w["Hkv"], w["L"], w["d"]
+    G = Hq // Hkv
+    # the first `pairs` (sequence, kv-head) groups: each group's G query heads read its K/V once
+    q = si.normal(seed, si.Q, (B, Hq, d))
+    kc = si.normal(seed, si.KCACHE, (B, L, Hkv, d))
+    vc = si.normal(seed, si.VCACHE, (B, L, Hkv, d))
+    rows = []
+    for p in range(pairs):
+        b, g = p // Hkv, p % Hkv
+        rows += [(b, g * G + j, 0) for j in range(G)]
+    rows = np.array(rows, np.int64)
+    t = time.perf_counter()
+    orc.attention_rows(q.reshape(B, 1, Hq, d), kc, vc, 1.0 / math.sqrt(d), rows, causal=False,
+                       kv_lens=np.full(B, L, np.int32), nthreads=threads)
+    dt = time.perf_counter() - t
+    return dt, pairs * L * d * 2 * 2
+
+
+def cpu_baseline_dec(seconds: float):
+    import oracle
+    orc = oracle.get()
+    threads = orc.hardware_threads()
+    dt, by = _oracle_dec(orc, 1, threads, DEC["seed"])
+    pairs = int(min(DEC["B"] * DEC["Hkv"], max(1, seconds / max(dt, 1e-3))))
+    dt, by = _oracle_dec(orc, pairs, threads, DEC["seed"])
+    return {"value": round(by / dt / 1e9, 3), "unit": "GB/s", "cores": threads, "kind": "oracle",
+            "sample": f"{pairs} of 64 (sequence, kv-head) groups of the decode workload, all 8 query heads each, "
+                      f"{dt:.1f} s on {threads} threads"}
+
+
+def run_reference(args):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    import oracle
+    orc = oracle.get()
+    threads = orc.hardware_threads()
+    per_step = max(0.5, args.cpu_seconds / max(1, args.steps))
+    dt0, _, n0 = _oracle_rows_fwd(orc, 64, threads, FWD["seed"])
+    rows = max(64, int(n0 * per_step / max(dt0, 1e-3)))
+    for _ in range(args.warmup):
+        _oracle_rows_fwd(orc, rows, threads, FWD["seed"])
+    tot_t, tot_f = 0.0, 0.0
+    for _ in range(args.steps):
+        dt, fl, _ = _oracle_rows_fwd(orc, rows, threads, FWD["seed"])
+        tot_t += dt
+        tot_f += fl
+    val = tot_f / tot_t / 1e12
+    line = {
+        "metric": METRIC, "value": round(val, 6), "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(1e3 * tot_t / args.steps, 3), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": "gqa_causal_8k: B=1, Hq=64, Hkv=8, N=8192, d=128, causal, layout [B,N,H,d]"},
+        "impl": "reference",
+        "cpu_baseline": {"value": round(val, 6), "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
+                         "sample": f"{rows} random causal rows per step (fp64 oracle, materialised rows)"},
+        "e2e": {"value": round(val, 6), "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="b200", choices=["b200", "reference"])
+    ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    ap.add_argument("--no-cpu", action="store_true", help="skip the CPU oracle baseline")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_device(args)
+
+
+if __name__ == "__main__":
+    main()

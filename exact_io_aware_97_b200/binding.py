@@ -1,0 +1,168 @@
+"""ctypes binding of libfa.so: the functions of include/fa.h under the same names.
+
+Argument marshalling only: pointers come from torch tensors (``data_ptr()``) or plain
+integers, the stream defaults to torch's current stream, and a non-OK status raises
+``FaError``.  Every step of the computation runs in the library's CUDA kernels; there is no
+fallback.  If libfa.so is missing this module raises on first use.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional
+
+PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(PKG, "libfa.so")
+
+FA_OK, FA_ERR_INVALID_ARG, FA_ERR_UNSUPPORTED, FA_ERR_WORKSPACE, FA_ERR_CUDA, FA_ERR_TIMEOUT = range(6)
+FA_BF16, FA_F32 = 0, 1
+
+EXPORTED = ("fa_fwd", "fa_fwd_workspace_size", "fa_decode", "fa_decode_workspace_size",
+            "fa_last_device_error", "fa_status_string", "fa_device_sm_count")
+
+
+class FaError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {status_string(status)} (status {status})")
+
+
+_lib: Optional[ctypes.CDLL] = None
+
+
+def load(path: str = LIB_PATH) -> ctypes.CDLL:
+    """Load libfa.so (once).  Raises if the CUDA library has not been built."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(path):
+        raise RuntimeError(f"libfa.so not found at {path}; build it with `python -m exact_io_aware_97_b200.build`")
+    L = ctypes.CDLL(path)
+    vp, i, f, sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
+    L.fa_fwd.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, i, f, i, vp, i, vp, sz, vp]
+    L.fa_fwd.restype = i
+    L.fa_fwd_workspace_size.argtypes = [i, i, i, i, i, i, i, i]
+    L.fa_fwd_workspace_size.restype = sz
+    L.fa_decode.argtypes = [vp, vp, vp, vp, vp, vp, i, i, i, i, i, f, i, vp, sz, vp]
+    L.fa_decode.restype = i
+    L.fa_decode_workspace_size.argtypes = [i, i, i, i, i]
+    L.fa_decode_workspace_size.restype = sz
+    L.fa_last_device_error.argtypes = [vp]
+    L.fa_last_device_error.restype = i
+    L.fa_status_string.argtypes = [i]
+    L.fa_status_string.restype = ctypes.c_char_p
+    L.fa_device_sm_count.argtypes = []
+    L.fa_device_sm_count.restype = i
+    _lib = L
+    return L
+
+
+def _ptr(x) -> Optional[int]:
+    if x is None:
+        return None
+    if isinstance(x, int):
+        return x or None
+    return x.data_ptr() or None
+
+
+def _stream(stream) -> Optional[int]:
+    if stream is None:
+        import torch
+        return torch.cuda.current_stream().cuda_stream or None
+    if isinstance(stream, int):
+        return stream or None
+    return stream.cuda_stream or None
+
+
+def _check(status: int, where: str) -> None:
+    if status != FA_OK:
+        raise FaError(status, where)
+
+
+def status_string(status: int) -> str:
+    return load().fa_status_string(int(status)).decode()
+
+
+def fa_fwd(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, d, scale, causal, cu_seqlens=None, in_dtype=FA_BF16,
+           workspace=None, workspace_bytes=0, stream=None) -> None:
+    st = load().fa_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), int(B), int(Hq), int(Hkv), int(Nq), int(Nk),
+                       int(d), float(scale), int(bool(causal)), _ptr(cu_seqlens), int(in_dtype), _ptr(workspace),
+                       int(workspace_bytes), _stream(stream))
+    _check(st, "fa_fwd")
+
+
+def fa_fwd_workspace_size(B, Hq, Hkv, Nq, Nk, d, in_dtype=FA_BF16, varlen=False) -> int:
+    return int(load().fa_fwd_workspace_size(int(B), int(Hq), int(Hkv), int(Nq), int(Nk), int(d), int(in_dtype),
+                                            int(bool(varlen))))
+
+
+def fa_decode(q, kcache, vcache, seqlens, o, lse, B, Hq, Hkv, Lmax, d, scale, split_len, workspace,
+              workspace_bytes, stream=None) -> None:
+    st = load().fa_decode(_ptr(q), _ptr(kcache), _ptr(vcache), _ptr(seqlens), _ptr(o), _ptr(lse), int(B), int(Hq),
+                          int(Hkv), int(Lmax), int(d), float(scale), int(split_len), _ptr(workspace),
+                          int(workspace_bytes), _stream(stream))
+    _check(st, "fa_decode")
+
+
+def fa_decode_workspace_size(B, Hq, Lmax, d, split_len) -> int:
+    return int(load().fa_decode_workspace_size(int(B), int(Hq), int(Lmax), int(d), int(split_len)))
+
+
+def fa_last_device_error(stream=None) -> int:
+    return int(load().fa_last_device_error(_stream(stream)))
+
+
+def fa_device_sm_count() -> int:
+    return int(load().fa_device_sm_count())
+
+
+# ------------------------------------------------------------------ tensor-level helpers
+def forward(q, k, v, causal=False, scale=None, cu_seqlens=None, out=None, lse=None, workspace=None, stream=None):
+    """O, lse for q [B,Nq,Hq,d] / k,v [B,Nk,Hkv,d] (or packed [total,H,d] with cu_seqlens).
+
+    bf16 inputs give bf16 O; fp32 inputs (fixed length) are rounded to bf16 on the device and
+    give fp32 O.  Outputs and workspace are allocated with torch unless passed in."""
+    import torch
+    varlen = cu_seqlens is not None
+    if varlen:
+        total, Hq, d = q.shape
+        Hkv = k.shape[1]
+        B, Nq, Nk = cu_seqlens.numel() - 1, total, total
+        lse_shape = (Hq, total)
+    else:
+        B, Nq, Hq, d = q.shape
+        Nk, Hkv = k.shape[1], k.shape[2]
+        lse_shape = (B, Hq, Nq)
+    in_dtype = FA_F32 if q.dtype == torch.float32 else FA_BF16
+    if scale is None:
+        scale = d ** -0.5
+    if out is None:
+        out = torch.empty(q.shape, dtype=torch.float32 if in_dtype == FA_F32 else torch.bfloat16, device=q.device)
+    if lse is None:
+        lse = torch.empty(lse_shape, dtype=torch.float32, device=q.device)
+    ws_bytes = fa_fwd_workspace_size(B, Hq, Hkv, Nq, Nk, d, in_dtype, varlen)
+    if ws_bytes and workspace is None:
+        workspace = torch.empty(ws_bytes, dtype=torch.uint8, device=q.device)
+    fa_fwd(q, k, v, out, lse, B, Hq, Hkv, Nq, Nk, d, scale, causal, cu_seqlens, in_dtype, workspace,
+           ws_bytes if workspace is not None else 0, stream)
+    return out, lse
+
+
+def decode(q, kcache, vcache, seqlens=None, scale=None, split_len=1024, out=None, lse=None, workspace=None,
+           stream=None):
+    """O [B,Hq,d], lse [B,Hq] for one query token per sequence over caches [B,Lmax,Hkv,d]."""
+    import torch
+    B, Hq, d = q.shape
+    Lmax, Hkv = kcache.shape[1], kcache.shape[2]
+    if scale is None:
+        scale = d ** -0.5
+    if out is None:
+        out = torch.empty((B, Hq, d), dtype=torch.bfloat16, device=q.device)
+    if lse is None:
+        lse = torch.empty((B, Hq), dtype=torch.float32, device=q.device)
+    ws_bytes = fa_decode_workspace_size(B, Hq, Lmax, d, split_len)
+    if workspace is None:
+        workspace = torch.empty(max(ws_bytes, 1), dtype=torch.uint8, device=q.device)
+    fa_decode(q, kcache, vcache, seqlens, out, lse, B, Hq, Hkv, Lmax, d, scale, split_len, workspace, ws_bytes,
+              stream)
+    return out, lse

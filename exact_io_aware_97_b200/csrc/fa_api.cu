@@ -1,0 +1,275 @@
+// Host side of the C ABI declared in include/fa.h: argument checks, TMA descriptors,
+// workspace carving and kernel launches.  No device memory is allocated here.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdint>
+#include <mutex>
+
+#include "../../include/fa.h"
+#include "fa_decode_sm100.cuh"
+#include "fa_fwd_sm100.cuh"
+
+namespace fa {
+
+// fp32 -> bf16 (round to nearest even), used when the forward is called with fp32 inputs.
+__global__ void cast_f32_bf16_kernel(const float* __restrict__ src, __nv_bfloat16* __restrict__ dst, size_t n) {
+  const size_t n4 = n / 4;
+  const size_t stride = (size_t)gridDim.x * blockDim.x;
+  for (size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x; i < n4; i += stride) {
+    const float4 x = reinterpret_cast<const float4*>(src)[i];
+    uint2 w;
+    w.x = pack_bf16x2(x.x, x.y);
+    w.y = pack_bf16x2(x.z, x.w);
+    reinterpret_cast<uint2*>(dst)[i] = w;
+  }
+  for (size_t i = n4 * 4 + (size_t)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += stride)
+    dst[i] = __float2bfloat16_rn(src[i]);
+}
+
+namespace {
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn get_encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(ptr);
+  });
+  return fn;
+}
+
+// [rows, heads, D] bf16 tensor (D innermost) seen as a 3-D map {D, heads, rows}; box of
+// 64 columns x 1 head x box_rows rows with the 128-byte swizzle.
+bool make_map(CUtensorMap* map, const void* base, int D, int heads, int64_t rows, int box_rows) {
+  EncodeTiledFn enc = get_encode_fn();
+  if (!enc) return false;
+  cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)heads, (cuuint64_t)rows};
+  cuuint64_t strides[2] = {(cuuint64_t)D * 2, (cuuint64_t)heads * D * 2};
+  cuuint32_t box[3] = {64, 1, (cuuint32_t)box_rows};
+  cuuint32_t estr[3] = {1, 1, 1};
+  return enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+int sm_count_cached() {
+  static int counts[64] = {0};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 0;
+  if (counts[dev] == 0) {
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
+    counts[dev] = n;
+  }
+  return counts[dev];
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+template <class K>
+cudaError_t set_smem(K kernel, int bytes) {
+  return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+}
+
+template <int D, bool F32>
+fa_status launch_fwd(const void* q, const void* k, const void* v, const FwdParams& prm, int64_t rows_q,
+                     int64_t rows_k, int units, cudaStream_t st) {
+  CUtensorMap mq, mk, mv;
+  if (!make_map(&mq, q, D, prm.Hq, rows_q, kBM) || !make_map(&mk, k, D, prm.Hkv, rows_k, kBN) ||
+      !make_map(&mv, v, D, prm.Hkv, rows_k, kBN))
+    return FA_ERR_CUDA;
+  auto kern = fa_fwd_kernel<D, F32>;
+  const int smem = FwdCfg<D>::kSmemBytes;
+  if (set_smem(kern, smem) != cudaSuccess) return FA_ERR_CUDA;
+  const int sms = sm_count_cached();
+  if (sms <= 0) return FA_ERR_CUDA;
+  const int grid = (units > 0) ? std::min(units, sms) : sms;
+  kern<<<grid, kFwdThreads, smem, st>>>(mq, mk, mv, prm);
+  return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+}
+
+template <int D>
+fa_status launch_decode(const void* kc, const void* vc, const DecParams& prm, cudaStream_t st) {
+  CUtensorMap mk, mv;
+  const int64_t rows = (int64_t)prm.B * prm.Lmax;
+  if (!make_map(&mk, kc, D, prm.Hkv, rows, kDecKeys) || !make_map(&mv, vc, D, prm.Hkv, rows, kDecKeys))
+    return FA_ERR_CUDA;
+  auto ks = fa_decode_split_kernel<D>;
+  const int smem = DecCfg<D>::kSmemBytes;
+  if (set_smem(ks, smem) != cudaSuccess) return FA_ERR_CUDA;
+  dim3 grid(prm.nsplit, prm.Hkv, prm.B);
+  ks<<<grid, kDecThreads, smem, st>>>(mk, mv, prm);
+  if (cudaGetLastError() != cudaSuccess) return FA_ERR_CUDA;
+  const int nbh = prm.B * prm.Hq;
+  fa_decode_combine_kernel<D><<<(nbh + 3) / 4, 128, 0, st>>>(prm);
+  return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+}
+
+}  // namespace
+}  // namespace fa
+
+using namespace fa;
+
+extern "C" {
+
+const char* fa_status_string(fa_status s) {
+  switch (s) {
+    case FA_OK: return "ok";
+    case FA_ERR_INVALID_ARG: return "invalid argument";
+    case FA_ERR_UNSUPPORTED: return "unsupported configuration";
+    case FA_ERR_WORKSPACE: return "workspace missing or too small";
+    case FA_ERR_CUDA: return "CUDA error";
+    case FA_ERR_TIMEOUT: return "device wait timed out";
+  }
+  return "unknown status";
+}
+
+int fa_device_sm_count(void) { return sm_count_cached(); }
+
+size_t fa_fwd_workspace_size(int B, int Hq, int Hkv, int Nq, int Nk, int d, fa_dtype in_dtype, int varlen) {
+  if (in_dtype != FA_F32 || varlen) return 0;
+  if (B <= 0 || Hq <= 0 || Hkv <= 0 || Nq < 0 || Nk < 0 || d <= 0) return 0;
+  const size_t nq = (size_t)B * Nq * Hq * d, nk = (size_t)B * Nk * Hkv * d;
+  return align_up(nq * 2, 256) + 2 * align_up(nk * 2, 256);
+}
+
+fa_status fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq, int Hkv, int Nq,
+                 int Nk, int d, float scale, int causal, const int32_t* cu_seqlens, fa_dtype in_dtype,
+                 void* workspace, size_t workspace_bytes, void* stream) {
+  if (!q || !k || !v || !o) return FA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o)) return FA_ERR_INVALID_ARG;
+  if (B < 0 || Hq <= 0 || Hkv <= 0 || Nq < 0 || Nk < 0) return FA_ERR_INVALID_ARG;
+  if (!(scale > 0.f) || !std::isfinite(scale)) return FA_ERR_INVALID_ARG;
+  if (in_dtype != FA_BF16 && in_dtype != FA_F32) return FA_ERR_INVALID_ARG;
+  if (Hq % Hkv != 0) return FA_ERR_UNSUPPORTED;
+  if (d != 64 && d != 128) return FA_ERR_UNSUPPORTED;
+  const bool varlen = cu_seqlens != nullptr;
+  if (varlen) {
+    if (Nq != Nk) return FA_ERR_INVALID_ARG;
+    if (in_dtype != FA_BF16) return FA_ERR_UNSUPPORTED;
+    if (B > kMaxVarlenB || (int64_t)Nq > (int64_t)kMaxVarlenT * kUnitRows) return FA_ERR_UNSUPPORTED;
+    if ((reinterpret_cast<uintptr_t>(cu_seqlens) & 3u) != 0) return FA_ERR_INVALID_ARG;
+  }
+  const int64_t rows_q = varlen ? (int64_t)Nq : (int64_t)B * Nq;
+  const int64_t rows_k = varlen ? (int64_t)Nk : (int64_t)B * Nk;
+  if (rows_q >= (int64_t(1) << 31) || rows_k >= (int64_t(1) << 31)) return FA_ERR_UNSUPPORTED;
+  if (B == 0 || Nq == 0) return FA_OK;
+
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const void *qb = q, *kb = k, *vb = v;
+  if (in_dtype == FA_F32) {
+    const size_t need = fa_fwd_workspace_size(B, Hq, Hkv, Nq, Nk, d, in_dtype, 0);
+    if (!workspace || workspace_bytes < need || !aligned16(workspace)) return FA_ERR_WORKSPACE;
+    const size_t nq = (size_t)rows_q * Hq * d, nk = (size_t)rows_k * Hkv * d;
+    uint8_t* w = static_cast<uint8_t*>(workspace);
+    __nv_bfloat16* q16 = reinterpret_cast<__nv_bfloat16*>(w);
+    __nv_bfloat16* k16 = reinterpret_cast<__nv_bfloat16*>(w + align_up(nq * 2, 256));
+    __nv_bfloat16* v16 = reinterpret_cast<__nv_bfloat16*>(w + align_up(nq * 2, 256) + align_up(nk * 2, 256));
+    const int sms = std::max(sm_count_cached(), 1);
+    cast_f32_bf16_kernel<<<sms * 4, 256, 0, st>>>(static_cast<const float*>(q), q16, nq);
+    if (nk > 0) {
+      cast_f32_bf16_kernel<<<sms * 4, 256, 0, st>>>(static_cast<const float*>(k), k16, nk);
+      cast_f32_bf16_kernel<<<sms * 4, 256, 0, st>>>(static_cast<const float*>(v), v16, nk);
+    }
+    if (cudaGetLastError() != cudaSuccess) return FA_ERR_CUDA;
+    qb = q16;
+    kb = k16;
+    vb = v16;
+  }
+
+  FwdParams prm{};
+  prm.o = o;
+  prm.lse = lse;
+  prm.cu = cu_seqlens;
+  prm.B = B;
+  prm.Hq = Hq;
+  prm.Hkv = Hkv;
+  prm.G = Hq / Hkv;
+  prm.Nq = Nq;
+  prm.Nk = Nk;
+  prm.causal = causal ? 1 : 0;
+  prm.tau = (float)((double)scale * 1.4426950408889634074);
+  prm.T = varlen ? 0 : (Nq + kUnitRows - 1) / kUnitRows;
+  const int64_t units64 = varlen ? 0 : (int64_t)prm.T * B * Hq;
+  if (units64 >= (int64_t(1) << 31)) return FA_ERR_UNSUPPORTED;
+  const int units = (int)units64;
+  const bool f32out = in_dtype == FA_F32;
+  // rows_k may be 0 (no keys); the map still needs a non-zero extent
+  const int64_t rk = std::max<int64_t>(rows_k, 1);
+  if (d == 64)
+    return f32out ? launch_fwd<64, true>(qb, kb, vb, prm, rows_q, rk, units, st)
+                  : launch_fwd<64, false>(qb, kb, vb, prm, rows_q, rk, units, st);
+  return f32out ? launch_fwd<128, true>(qb, kb, vb, prm, rows_q, rk, units, st)
+                : launch_fwd<128, false>(qb, kb, vb, prm, rows_q, rk, units, st);
+}
+
+size_t fa_decode_workspace_size(int B, int Hq, int Lmax, int d, int split_len) {
+  if (B <= 0 || Hq <= 0 || Lmax <= 0 || d <= 0 || split_len <= 0) return 0;
+  const size_t ns = (size_t)((Lmax + split_len - 1) / split_len);
+  const size_t parts = (size_t)B * Hq * ns;
+  return align_up(parts * d * 4, 256) + align_up(parts * 2 * 4, 256);
+}
+
+fa_status fa_decode(const void* q, const void* kcache, const void* vcache, const int32_t* seqlens, void* o,
+                    float* lse, int B, int Hq, int Hkv, int Lmax, int d, float scale, int split_len,
+                    void* workspace, size_t workspace_bytes, void* stream) {
+  if (!q || !kcache || !vcache || !o) return FA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(kcache) || !aligned16(vcache) || !aligned16(o)) return FA_ERR_INVALID_ARG;
+  if (B < 0 || Hq <= 0 || Hkv <= 0 || Lmax <= 0 || split_len <= 0) return FA_ERR_INVALID_ARG;
+  if (!(scale > 0.f) || !std::isfinite(scale)) return FA_ERR_INVALID_ARG;
+  if (seqlens && (reinterpret_cast<uintptr_t>(seqlens) & 3u) != 0) return FA_ERR_INVALID_ARG;
+  if (Hq % Hkv != 0) return FA_ERR_UNSUPPORTED;
+  if (Hq / Hkv > 16) return FA_ERR_UNSUPPORTED;
+  if (d != 64 && d != 128) return FA_ERR_UNSUPPORTED;
+  if (split_len % kDecKeys != 0) return FA_ERR_UNSUPPORTED;
+  if ((int64_t)B * Lmax >= (int64_t(1) << 31)) return FA_ERR_UNSUPPORTED;
+  if (B == 0) return FA_OK;
+  const int nsplit = (Lmax + split_len - 1) / split_len;
+  if (nsplit > 65535 || Hkv > 65535 || B > 65535) return FA_ERR_UNSUPPORTED;
+  const size_t need = fa_decode_workspace_size(B, Hq, Lmax, d, split_len);
+  if (!workspace || workspace_bytes < need || !aligned16(workspace)) return FA_ERR_WORKSPACE;
+  const size_t parts = (size_t)B * Hq * nsplit;
+  DecParams prm{};
+  prm.q = static_cast<const __nv_bfloat16*>(q);
+  prm.seqlens = seqlens;
+  prm.o = static_cast<__nv_bfloat16*>(o);
+  prm.lse = lse;
+  prm.ws_acc = static_cast<float*>(workspace);
+  prm.ws_ml = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + align_up(parts * d * 4, 256));
+  prm.B = B;
+  prm.Hq = Hq;
+  prm.Hkv = Hkv;
+  prm.G = Hq / Hkv;
+  prm.Lmax = Lmax;
+  prm.split_len = split_len;
+  prm.nsplit = nsplit;
+  prm.tau = (float)((double)scale * 1.4426950408889634074);
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  return d == 64 ? launch_decode<64>(kcache, vcache, prm, st) : launch_decode<128>(kcache, vcache, prm, st);
+}
+
+fa_status fa_last_device_error(void* stream) {
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (cudaStreamSynchronize(st) != cudaSuccess) return FA_ERR_CUDA;
+  unsigned int w = 0;
+  if (cudaMemcpyFromSymbol(&w, g_error_word, sizeof(w)) != cudaSuccess) return FA_ERR_CUDA;
+  if (w != 0) {
+    const unsigned int zero = 0;
+    if (cudaMemcpyToSymbol(g_error_word, &zero, sizeof(zero)) != cudaSuccess) return FA_ERR_CUDA;
+    return FA_ERR_TIMEOUT;
+  }
+  return FA_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,548 @@
+// Forward attention kernel for sm_100a.
+//
+// The method ("FlashAttention notes", sections 3-4; "LLM basics: from Attention to
+// FlashAttention", chapter 3 sections 2 and 5): a tile of query rows stays on chip while
+// tiles of K and V stream past it; for each K/V tile the scores S = Q K^T are formed on
+// chip, the running row max m and row sum l are updated with
+//   m_new = max(m_old, rowmax(S)),  l_new = e^(m_old - m_new) l_old + sum_j e^(s_j - m_new),
+// the output accumulator is rescaled by the same factor and P V is added to it.  Only O
+// and the per-row logsumexp are written to device memory.
+//
+// B200 mapping (one persistent CTA per SM, 320 threads):
+//   warps 0-3  softmax for query tile 0 (thread = row), then its epilogue
+//   warps 4-7  softmax for query tile 1
+//   warp  8    tcgen05.mma issuer (one thread) and TMEM owner
+//   warp  9    TMA producer (one thread)
+// A work unit is 256 query rows (two 128-row tiles) of one (sequence, query head).  Units
+// are ordered longest-first (causal cost grows with the query tile index) and dealt to
+// CTAs in a snake order.  K and V tiles (128 keys each) flow through a shared-memory ring
+// of full/empty mbarriers.  TMEM (512 columns): S0 | S1 (128 fp32 columns each, P is
+// written back over the first 64 columns of its S as packed bf16) | O0 | O1 (d columns).
+// The MMA order S0(j+1) after O0 += P0(j) V(j) and S1(j+1) after O1 += P1(j) V(j) lets the
+// tensor core work on one tile while the softmax warps work on the other.
+//
+// Scores are handled in base 2: t = s * scale * log2(e), p = 2^(t - m).  The output is
+// rescaled lazily: the reference max m only moves when the tile max exceeds it by more than
+// 8 (a factor 256), which is exact because O and l always share the same reference
+// ("LLM basics", chapter 3 section 1: subtracting any constant leaves softmax unchanged).
+#pragma once
+
+#include "fa_device.cuh"
+
+namespace fa {
+
+struct FwdParams {
+  void* o;
+  float* lse;
+  const int32_t* cu;  // varlen offsets [B+1] or null
+  int B, Hq, Hkv, G, Nq, Nk;
+  int causal;
+  float tau;  // scale * log2(e)
+  int T;      // fixed length: 256-row units per (sequence, head)
+};
+
+constexpr int kBM = 128;        // query rows per tile
+constexpr int kBN = 128;        // keys per K/V tile
+constexpr int kUnitRows = 256;  // two query tiles per work unit
+constexpr int kFwdThreads = 320;
+constexpr int kMaxVarlenB = 1024;
+constexpr int kMaxVarlenT = 1024;
+constexpr float kRescaleThreshold = 8.0f;
+
+template <int D>
+struct FwdCfg {
+  static constexpr int kTileBytes = kBM * D * 2;  // one 128 x D bf16 tile
+  static constexpr int kChunkBytes = kBM * 128;   // one 128-row x 64-column swizzle panel
+  static constexpr int kStages = (D == 128) ? 4 : 8;
+  static constexpr int kQBytes = 2 * kTileBytes;
+  static constexpr int kRingBytes = kStages * kTileBytes;
+  static constexpr int kNumBars = 2 + 2 * kStages + 8;
+  static constexpr int kBarBytes = kNumBars * 8 + 16;
+  static constexpr int kSchedBytes = kMaxVarlenB * 2 + kMaxVarlenT * 4 + 16;
+  static constexpr int kSmemBytes = 1024 + kQBytes + kRingBytes + kBarBytes + kSchedBytes;
+  static constexpr uint32_t kTmemCols = 512;
+  static constexpr uint32_t kColO = 256;
+};
+
+// Geometry of one work unit as every role sees it.
+struct Unit {
+  int b, h, kvh;
+  int q_start, k_start;  // first row of the sequence in q/o and in k/v
+  int nq, nk;
+  int row0;   // first query row of the unit within the sequence
+  int n[2];   // K/V tiles each query tile attends to (0: tile empty or sees no key)
+  int valid[2];
+  int nmax;
+};
+
+struct SchedShared {
+  int T;          // number of levels (query-tile indices)
+  int U;          // total units
+  uint16_t* sigma;  // varlen: sequences sorted by tile count, descending
+  int* cnt;         // varlen: cnt[t] = number of sequences with more than t unit rows-tiles
+};
+
+// Walks the units of one CTA in increasing order.
+struct UnitWalker {
+  int level = 0;
+  int level_start = 0;
+};
+
+__device__ __forceinline__ int kv_tiles_for(int last_row, int nq, int nk, int causal) {
+  int kv_end = nk;
+  if (causal) kv_end = min(nk, last_row + (nk - nq) + 1);
+  if (kv_end <= 0) return 0;
+  return (kv_end + kBN - 1) / kBN;
+}
+
+__device__ __forceinline__ void decode_unit(const FwdParams& p, const SchedShared& s, UnitWalker& w, int u,
+                                            Unit& out) {
+  int b, t, h;
+  if (p.cu == nullptr) {
+    const int per_level = p.B * p.Hq;
+    const int level = u / per_level;
+    const int off = u - level * per_level;
+    b = off / p.Hq;
+    h = off - b * p.Hq;
+    t = s.T - 1 - level;
+    out.q_start = b * p.Nq;
+    out.k_start = b * p.Nk;
+    out.nq = p.Nq;
+    out.nk = p.Nk;
+  } else {
+    for (;;) {
+      const int sz = s.cnt[s.T - 1 - w.level] * p.Hq;
+      if (u < w.level_start + sz) break;
+      w.level_start += sz;
+      ++w.level;
+    }
+    const int off = u - w.level_start;
+    const int r = off / p.Hq;
+    h = off - r * p.Hq;
+    b = s.sigma[r];
+    t = s.T - 1 - w.level;
+    const int c0 = __ldg(p.cu + b), c1 = __ldg(p.cu + b + 1);
+    out.q_start = c0;
+    out.k_start = c0;
+    out.nq = c1 - c0;
+    out.nk = c1 - c0;
+  }
+  out.b = b;
+  out.h = h;
+  out.kvh = h / p.G;
+  out.row0 = t * kUnitRows;
+  for (int i = 0; i < 2; ++i) {
+    const int r0 = out.row0 + i * kBM;
+    out.valid[i] = r0 < out.nq;
+    out.n[i] = out.valid[i] ? kv_tiles_for(min(r0 + kBM - 1, out.nq - 1), out.nq, out.nk, p.causal) : 0;
+  }
+  out.nmax = max(out.n[0], out.n[1]);
+}
+
+// The u-th unit handled by CTA c (snake order over rounds of gridDim.x units); -1 when done.
+struct UnitIter {
+  int round = 0;
+  __device__ __forceinline__ int next(int U) {
+    const int G = gridDim.x, c = blockIdx.x;
+    for (;;) {
+      if (round * G >= U) return -1;
+      const int u = round * G + ((round & 1) ? (G - 1 - c) : c);
+      ++round;
+      if (u < U) return u;
+    }
+  }
+};
+
+template <int D, bool OUT_F32>
+__global__ void __launch_bounds__(kFwdThreads, 1)
+    fa_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                  const __grid_constant__ CUtensorMap tmV, const FwdParams p) {
+  using C = FwdCfg<D>;
+  constexpr int NS = C::kStages;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sQ = smem;
+  uint8_t* sRing = smem + C::kQBytes;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sRing + C::kRingBytes);
+  uint64_t* q_full = bars + 0;
+  uint64_t* q_empty = bars + 1;
+  uint64_t* full = bars + 2;
+  uint64_t* empty = bars + 2 + NS;
+  uint64_t* s_full = bars + 2 + 2 * NS;  // [2]
+  uint64_t* p_full = s_full + 2;         // [2]
+  uint64_t* pv_done = p_full + 2;        // [2]
+  uint64_t* o_free = pv_done + 2;        // [2]
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + C::kNumBars);
+  int* sched_misc = reinterpret_cast<int*>(tmem_slot + 2);  // [0] = T, [1] = total tiles
+  uint8_t* sched_mem = reinterpret_cast<uint8_t*>(bars) + C::kBarBytes;
+  uint16_t* sigma = reinterpret_cast<uint16_t*>(sched_mem);
+  int* cnt = reinterpret_cast<int*>(sched_mem + kMaxVarlenB * 2);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    mbar_init(q_full, 1);
+    mbar_init(q_empty, 1);
+    for (int s = 0; s < NS; ++s) {
+      mbar_init(full + s, 1);
+      mbar_init(empty + s, 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(s_full + i, 1);
+      mbar_init(p_full + i, kBM);
+      mbar_init(pv_done + i, 1);
+      mbar_init(o_free + i, kBM);
+    }
+    sched_misc[0] = 0;
+    sched_misc[1] = 0;
+    fence_barrier_init();
+  }
+  if (warp == 9 && lane == 0) {
+    prefetch_tensormap(&tmQ);
+    prefetch_tensormap(&tmK);
+    prefetch_tensormap(&tmV);
+  }
+  if (warp == 8) {
+    tmem_alloc(tmem_slot, C::kTmemCols);
+    tmem_relinquish();
+  }
+
+  // ---- schedule: fixed length is arithmetic; varlen sorts sequences by tile count
+  SchedShared sch;
+  sch.sigma = sigma;
+  sch.cnt = cnt;
+  if (p.cu == nullptr) {
+    sch.T = p.T;
+    sch.U = p.T * p.B * p.Hq;
+    __syncthreads();
+  } else {
+    __syncthreads();  // sched_misc initialised
+    for (int b = threadIdx.x; b < p.B; b += blockDim.x) {
+      const int len = __ldg(p.cu + b + 1) - __ldg(p.cu + b);
+      const int nt = len > 0 ? (len + kUnitRows - 1) / kUnitRows : 0;
+      atomicMax(&sched_misc[0], nt);
+      atomicAdd(&sched_misc[1], nt);
+    }
+    __syncthreads();
+    const int T = min(sched_misc[0], kMaxVarlenT);
+    for (int b = threadIdx.x; b < p.B; b += blockDim.x) {
+      const int lb = __ldg(p.cu + b + 1) - __ldg(p.cu + b);
+      const int nb = lb > 0 ? (lb + kUnitRows - 1) / kUnitRows : 0;
+      int rank = 0;
+      for (int b2 = 0; b2 < p.B; ++b2) {
+        const int l2 = __ldg(p.cu + b2 + 1) - __ldg(p.cu + b2);
+        const int n2 = l2 > 0 ? (l2 + kUnitRows - 1) / kUnitRows : 0;
+        rank += (n2 > nb) || (n2 == nb && b2 < b);
+      }
+      sigma[rank] = (uint16_t)b;
+    }
+    for (int t = threadIdx.x; t < T; t += blockDim.x) {
+      int c = 0;
+      for (int b2 = 0; b2 < p.B; ++b2) {
+        const int l2 = __ldg(p.cu + b2 + 1) - __ldg(p.cu + b2);
+        const int n2 = l2 > 0 ? (l2 + kUnitRows - 1) / kUnitRows : 0;
+        c += n2 > t;
+      }
+      cnt[t] = c;
+    }
+    __syncthreads();
+    sch.T = T;
+    sch.U = sched_misc[1] * p.Hq;
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 9) {
+    // ================================================================ TMA producer
+    if (lane == 0) {
+      const uint64_t kv_policy = policy_evict_last();
+      uint32_t g = 0, qcount = 0;
+      UnitIter it;
+      UnitWalker wk;
+      bool ok = true;
+      for (int u = it.next(sch.U); u >= 0 && ok; u = it.next(sch.U)) {
+        Unit un;
+        decode_unit(p, sch, wk, u, un);
+        if (qcount > 0 && !mbar_wait(q_empty, (qcount - 1) & 1)) break;
+        const int ntile = un.valid[1] ? 2 : 1;
+        mbar_arrive_expect_tx(q_full, ntile * C::kTileBytes);
+        for (int i = 0; i < ntile; ++i)
+          for (int c = 0; c < D / 64; ++c)
+            tma_load_3d(sQ + i * C::kTileBytes + c * C::kChunkBytes, &tmQ, c * 64, un.h,
+                        un.q_start + un.row0 + i * kBM, q_full);
+        for (int j = 0; j < un.nmax && ok; ++j) {
+          for (int kv = 0; kv < 2; ++kv) {
+            const uint32_t slot = g % NS;
+            if (g >= (uint32_t)NS && !mbar_wait(empty + slot, ((g / NS) - 1) & 1)) {
+              ok = false;
+              break;
+            }
+            mbar_arrive_expect_tx(full + slot, C::kTileBytes);
+            for (int c = 0; c < D / 64; ++c)
+              tma_load_3d_hint(sRing + slot * C::kTileBytes + c * C::kChunkBytes, kv ? &tmV : &tmK, c * 64,
+                               un.kvh, un.k_start + j * kBN, full + slot, kv_policy);
+            ++g;
+          }
+        }
+        ++qcount;
+      }
+    }
+    __syncwarp();
+  } else if (warp == 8) {
+    // ================================================================ MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t idS = idesc_bf16_f32(kBM, kBN, false);
+      constexpr uint32_t idPV = idesc_bf16_f32(kBM, D, true);
+      const uint32_t qbase = smem_u32(sQ);
+      const uint32_t rbase = smem_u32(sRing);
+      uint32_t g = 0, qcount = 0;
+      uint32_t pcnt[2] = {0, 0}, ounits[2] = {0, 0};
+      UnitIter it;
+      UnitWalker wk;
+      bool ok = true;
+
+      auto issue_S = [&](int i, uint32_t slot) {
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = (kk >> 2) * C::kChunkBytes + (kk & 3) * 32;
+          const uint64_t a = smem_desc_sw128(qbase + i * C::kTileBytes + off, 16, 1024);
+          const uint64_t bd = smem_desc_sw128(rbase + slot * C::kTileBytes + off, 16, 1024);
+          umma_ss(tmem + i * kBN, a, bd, idS, kk > 0 ? 1u : 0u);
+        }
+      };
+      auto issue_PV = [&](int i, uint32_t slot, bool acc) {
+#pragma unroll
+        for (int kk = 0; kk < kBN / 16; ++kk) {
+          const uint64_t bd = smem_desc_sw128(rbase + slot * C::kTileBytes + kk * 16 * 128, C::kChunkBytes, 1024);
+          umma_ts(tmem + C::kColO + i * D, tmem + i * kBN + kk * 8, bd, idPV, (acc || kk > 0) ? 1u : 0u);
+        }
+      };
+      auto wait_full = [&](uint32_t gi) -> bool {
+        if (!mbar_wait(full + (gi % NS), (gi / NS) & 1)) return false;
+        tc_fence_after();
+        return true;
+      };
+      auto pv_step = [&](int i, int j, uint32_t vslot) -> bool {
+        if (j == 0 && ounits[i] > 0 && !mbar_wait(o_free + i, (ounits[i] - 1) & 1)) return false;
+        if (!mbar_wait(p_full + i, pcnt[i] & 1)) return false;
+        ++pcnt[i];
+        tc_fence_after();
+        issue_PV(i, vslot, j > 0);
+        umma_commit(pv_done + i);
+        return true;
+      };
+
+      for (int u = it.next(sch.U); u >= 0 && ok; u = it.next(sch.U)) {
+        Unit un;
+        decode_unit(p, sch, wk, u, un);
+        if (!mbar_wait(q_full, qcount & 1)) break;
+        tc_fence_after();
+        const int nmax = un.nmax;
+        if (nmax == 0) {
+          umma_commit(q_empty);
+          ++qcount;
+          continue;
+        }
+        // prologue: S_i(0)
+        if (!wait_full(g)) break;
+        for (int i = 0; i < 2; ++i)
+          if (un.n[i] > 0) {
+            issue_S(i, g % NS);
+            umma_commit(s_full + i);
+          }
+        umma_commit(empty + (g % NS));
+        if (nmax == 1) umma_commit(q_empty);
+        for (int j = 0; j < nmax && ok; ++j) {
+          const uint32_t gv = g + 2 * j + 1;
+          const uint32_t gk = g + 2 * j + 2;
+          if (!wait_full(gv)) { ok = false; break; }
+          if (j < un.n[0] && !pv_step(0, j, gv % NS)) { ok = false; break; }
+          if (j + 1 < nmax) {
+            if (!wait_full(gk)) { ok = false; break; }
+            if (j + 1 < un.n[0]) {
+              issue_S(0, gk % NS);
+              umma_commit(s_full + 0);
+            }
+          }
+          if (j < un.n[1] && !pv_step(1, j, gv % NS)) { ok = false; break; }
+          umma_commit(empty + (gv % NS));
+          if (j + 1 < nmax) {
+            if (j + 1 < un.n[1]) {
+              issue_S(1, gk % NS);
+              umma_commit(s_full + 1);
+            }
+            umma_commit(empty + (gk % NS));
+            if (j + 2 == nmax) umma_commit(q_empty);
+          }
+        }
+        g += 2 * nmax;
+        ++qcount;
+        for (int i = 0; i < 2; ++i)
+          if (un.n[i] > 0) ++ounits[i];
+      }
+    }
+    __syncwarp();
+  } else {
+    // ================================================================ softmax + epilogue
+    const int i = warp >> 2;            // query tile of this warpgroup
+    const int r = threadIdx.x & 127;    // row within the tile = TMEM lane
+    const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
+    const uint32_t tS = tmem + lane_off + i * kBN;
+    const uint32_t tO = tmem + lane_off + C::kColO + i * D;
+    const float tau = p.tau;
+    uint32_t scnt = 0, pvcnt = 0;
+    UnitIter it;
+    UnitWalker wk;
+    bool ok = true;
+
+    for (int u = it.next(sch.U); u >= 0 && ok; u = it.next(sch.U)) {
+      Unit un;
+      decode_unit(p, sch, wk, u, un);
+      const int my_valid = i ? un.valid[1] : un.valid[0];
+      if (!my_valid) continue;
+      const int n = i ? un.n[1] : un.n[0];
+      const int row = un.row0 + i * kBM + r;                       // row within the sequence
+      const int warp_row_min = un.row0 + i * kBM + (warp & 3) * 32;
+      const int diag = un.nk - un.nq;                              // causal offset
+      float m_ref = -INFINITY, l = 0.f;
+
+      for (int j = 0; j < n; ++j) {
+        if (!mbar_wait(s_full + i, scnt & 1)) { ok = false; break; }
+        ++scnt;
+        tc_fence_after();
+        uint32_t sv[4][32];
+#pragma unroll
+        for (int c = 0; c < 4; ++c) tmem_ld32(tS + 32 * c, sv[c]);
+        tmem_wait_ld();
+        float s[128];
+#pragma unroll
+        for (int c = 0; c < 128; ++c) s[c] = __uint_as_float(sv[c >> 5][c & 31]);
+
+        const int key0 = j * kBN;
+        const bool need_mask = (key0 + kBN > un.nk) || (p.causal && key0 + kBN - 1 > warp_row_min + diag);
+        if (need_mask) {
+          int lim = un.nk - key0;
+          if (p.causal) lim = min(lim, row + diag + 1 - key0);
+#pragma unroll
+          for (int c = 0; c < 128; ++c)
+            if (c >= lim) s[c] = -INFINITY;
+        }
+        float mx0 = s[0], mx1 = s[1], mx2 = s[2], mx3 = s[3];
+#pragma unroll
+        for (int c = 4; c < 128; c += 4) {
+          mx0 = fmaxf(mx0, s[c]);
+          mx1 = fmaxf(mx1, s[c + 1]);
+          mx2 = fmaxf(mx2, s[c + 2]);
+          mx3 = fmaxf(mx3, s[c + 3]);
+        }
+        const float m_tile = fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3)) * tau;
+        const float m_new = fmaxf(m_ref, m_tile);
+        const bool need = m_new - m_ref > kRescaleThreshold;  // false when both are -inf
+        const bool warp_need = __any_sync(0xffffffffu, need);
+        const float alpha = need ? ex2_approx(m_ref - m_new) : 1.f;
+        if (need) m_ref = m_new;
+        l *= alpha;
+        // P = 2^(t - m_ref), written as packed bf16 over the first 64 columns of S.
+        const float ms = (m_ref == -INFINITY) ? 0.f : m_ref;
+        float ls0 = 0.f, ls1 = 0.f;
+#pragma unroll
+        for (int half = 0; half < 2; ++half) {
+          uint32_t pk[32];
+#pragma unroll
+          for (int c = 0; c < 32; ++c) {
+            const float p0 = ex2_approx(fmaf(s[64 * half + 2 * c], tau, -ms));
+            const float p1 = ex2_approx(fmaf(s[64 * half + 2 * c + 1], tau, -ms));
+            ls0 += p0;
+            ls1 += p1;
+            pk[c] = pack_bf16x2(p0, p1);
+          }
+          tmem_st32(tS + 32 * half, pk);
+        }
+        l += ls0 + ls1;
+        if (warp_need && j > 0) {
+          // O holds P V up to tile j-1 (complete: S(j) was committed after that product);
+          // bring it to the new reference max.
+          if (!mbar_wait(pv_done + i, (pvcnt + j - 1) & 1)) { ok = false; break; }
+          tc_fence_after();
+#pragma unroll
+          for (int c = 0; c < D / 32; ++c) {
+            uint32_t ov[32];
+            tmem_ld32(tO + 32 * c, ov);
+            tmem_wait_ld();
+#pragma unroll
+            for (int e = 0; e < 32; ++e) ov[e] = __float_as_uint(__uint_as_float(ov[e]) * alpha);
+            tmem_st32(tO + 32 * c, ov);
+          }
+        }
+        tmem_wait_st();
+        tc_fence_before();
+        mbar_arrive(p_full + i);
+      }
+      if (!ok) break;
+
+      // ---- epilogue: O / l, lse
+      if (n > 0) {
+        if (!mbar_wait(pv_done + i, (pvcnt + n - 1) & 1)) { ok = false; break; }
+        tc_fence_after();
+      }
+      pvcnt += n;
+      const bool row_ok = row < un.nq;
+      const float inv_l = l > 0.f ? 1.f / l : 0.f;
+      const size_t orow = ((size_t)(un.q_start + row) * p.Hq + un.h) * D;
+#pragma unroll
+      for (int c = 0; c < D / 32; ++c) {
+        uint32_t ov[32];
+        if (n > 0) {
+          tmem_ld32(tO + 32 * c, ov);
+          tmem_wait_ld();
+        } else {
+#pragma unroll
+          for (int e = 0; e < 32; ++e) ov[e] = 0u;
+        }
+        if (row_ok) {
+          if (OUT_F32) {
+            float4* dst = reinterpret_cast<float4*>(reinterpret_cast<float*>(p.o) + orow + 32 * c);
+#pragma unroll
+            for (int e = 0; e < 8; ++e)
+              dst[e] = make_float4(__uint_as_float(ov[4 * e]) * inv_l, __uint_as_float(ov[4 * e + 1]) * inv_l,
+                                   __uint_as_float(ov[4 * e + 2]) * inv_l, __uint_as_float(ov[4 * e + 3]) * inv_l);
+          } else {
+            uint4* dst = reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(p.o) + orow + 32 * c);
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              uint4 w;
+              w.x = pack_bf16x2(__uint_as_float(ov[8 * e + 0]) * inv_l, __uint_as_float(ov[8 * e + 1]) * inv_l);
+              w.y = pack_bf16x2(__uint_as_float(ov[8 * e + 2]) * inv_l, __uint_as_float(ov[8 * e + 3]) * inv_l);
+              w.z = pack_bf16x2(__uint_as_float(ov[8 * e + 4]) * inv_l, __uint_as_float(ov[8 * e + 5]) * inv_l);
+              w.w = pack_bf16x2(__uint_as_float(ov[8 * e + 6]) * inv_l, __uint_as_float(ov[8 * e + 7]) * inv_l);
+              dst[e] = w;
+            }
+          }
+        }
+      }
+      if (row_ok && p.lse != nullptr) {
+        const float v = l > 0.f ? (m_ref + log2f(l)) * kLn2 : -INFINITY;
+        const size_t li = (p.cu != nullptr) ? (size_t)un.h * p.Nq + un.q_start + row
+                                             : ((size_t)un.b * p.Hq + un.h) * p.Nq + row;
+        p.lse[li] = v;
+      }
+      if (n > 0) {
+        tc_fence_before();
+        mbar_arrive(o_free + i);
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 8) {
+    tc_fence_after();
+    tmem_dealloc(tmem, C::kTmemCols);
+  }
+}
+
+}  // namespace fa

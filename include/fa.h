@@ -1,0 +1,117 @@
+/* Exact IO-aware attention for NVIDIA B200 (sm_100a): C ABI.
+ *
+ * Two operations, both computing exactly O = softmax(Q K^T * scale) V and the per-row
+ * logsumexp, tile by tile with the online-softmax running max m and sum l, so the N x N
+ * score and probability matrices never reach device memory:
+ *
+ *   fa_fwd     the tiled forward ("FlashAttention notes", section 3 "Tiling" and section 4
+ *              "Online Softmax": m_new = max(m1, m2), l_new = e^(m1-m_new) l1 + e^(m2-m_new) l2;
+ *              "LLM basics: from Attention to FlashAttention", chapter 3 section 5), with
+ *              causal masking (same tutorial, chapter 1 section 7), grouped-query heads
+ *              (chapter 2 section 7) and variable-length packed batches ("FlashAttention-3
+ *              (FA-3)", section 2 feature table: MQA, GQA, variable-length).
+ *   fa_decode  single-token decode over a KV cache, split along the cache; the partial
+ *              results are merged with the same m/l rule ("FlashAttention-3 (FA-3)",
+ *              section 4 "FlashDecoding"; "FlashAttention notes", section 4).
+ *
+ * Conventions for every entry point:
+ *   - All tensor pointers are DEVICE pointers owned by the caller.  The library never
+ *     allocates or frees device memory and never synchronises, except in
+ *     fa_last_device_error.  Every launch is asynchronous on `stream` (a cudaStream_t
+ *     passed as void*; NULL is the legacy default stream).
+ *   - Tensors are contiguous with the head dimension d innermost.  bf16 is IEEE bfloat16.
+ *   - Arguments are validated on the host before anything is launched; a rejected call
+ *     returns FA_ERR_INVALID_ARG or FA_ERR_UNSUPPORTED and touches no memory.
+ *   - A failed launch returns FA_ERR_CUDA.  A device-side wait that exceeded its time
+ *     limit (it never should) is recorded on the device and reported by
+ *     fa_last_device_error as FA_ERR_TIMEOUT; the kernel then returns instead of hanging.
+ */
+#ifndef FA_H
+#define FA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define FA_EXPORT __attribute__((visibility("default")))
+#else
+#define FA_EXPORT
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  FA_OK = 0,
+  FA_ERR_INVALID_ARG = 1, /* null/misaligned pointer, bad size, bad scale */
+  FA_ERR_UNSUPPORTED = 2, /* valid but not implemented (e.g. d not in {64, 128}) */
+  FA_ERR_WORKSPACE = 3,   /* workspace missing or smaller than the *_workspace_size() value */
+  FA_ERR_CUDA = 4,        /* a CUDA runtime/driver call failed */
+  FA_ERR_TIMEOUT = 5      /* a device wait gave up (reported by fa_last_device_error) */
+} fa_status;
+
+typedef enum { FA_BF16 = 0, FA_F32 = 1 } fa_dtype;
+
+/* Forward attention.
+ *
+ * Fixed length (cu_seqlens == NULL):
+ *   q [B, Nq, Hq, d], k and v [B, Nk, Hkv, d], o [B, Nq, Hq, d], lse [B, Hq, Nq].
+ * Variable length (cu_seqlens != NULL, device int32 [B+1], cu_seqlens[0] = 0, non-decreasing):
+ *   Nq == Nk == total packed rows; q and o [total, Hq, d], k and v [total, Hkv, d],
+ *   lse [Hq, total]; sequence b owns rows [cu_seqlens[b], cu_seqlens[b+1]) of q, k and v and
+ *   attends only within itself.  The caller guarantees cu_seqlens[B] <= total (it is read
+ *   on the device only).  B <= 1024.
+ *
+ * in_dtype FA_BF16: q, k, v, o are bf16.  FA_F32: q, k, v are fp32, rounded to bf16 (nearest
+ *   even) into the workspace first, and o is written as fp32; fixed length only.
+ * Accumulation is fp32; P is rounded to bf16 before the P*V product.
+ * scale: the score multiplier, > 0 (1/sqrt(d) in "LLM basics", chapter 1 section 3).
+ * causal: query i of a sequence with nq queries and nk keys sees keys j <= i + nk - nq
+ *   (bottom-right aligned; the usual lower triangle when nq == nk).  A row that sees no
+ *   key gets o = 0 and lse = -inf.
+ * lse: natural-log logsumexp of the scaled scores, fp32; may be NULL.
+ * Hq must be a multiple of Hkv; query head h uses key/value head h / (Hq / Hkv).
+ * d must be 64 or 128.  q, k, v, o must be 16-byte aligned.
+ * workspace: device memory of at least fa_fwd_workspace_size(...) bytes (may be NULL when
+ *   that size is 0).
+ */
+FA_EXPORT fa_status fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq, int Hkv,
+                 int Nq, int Nk, int d, float scale, int causal, const int32_t* cu_seqlens, fa_dtype in_dtype,
+                 void* workspace, size_t workspace_bytes, void* stream);
+
+FA_EXPORT size_t fa_fwd_workspace_size(int B, int Hq, int Hkv, int Nq, int Nk, int d, fa_dtype in_dtype, int varlen);
+
+/* Split-KV decode: one query token per sequence against its KV cache.
+ *
+ * q [B, Hq, d] bf16; kcache and vcache [B, Lmax, Hkv, d] bf16; o [B, Hq, d] bf16;
+ * lse [B, Hq] fp32 (may be NULL); seqlens: device int32 [B] with 0 <= seqlens[b] <= Lmax,
+ * or NULL meaning every sequence holds Lmax tokens.  Sequence b attends (non-causally) to
+ * cache rows j < seqlens[b]; an empty sequence gets o = 0 and lse = -inf.
+ * The cache is cut into splits of split_len rows (a multiple of 64); each split's partial
+ * (m, l, unnormalised acc) goes to the workspace and a second kernel merges them with the
+ * m/l rule.  Hq / Hkv <= 16.  d must be 64 or 128.  Pointers 16-byte aligned.
+ */
+FA_EXPORT fa_status fa_decode(const void* q, const void* kcache, const void* vcache, const int32_t* seqlens, void* o,
+                    float* lse, int B, int Hq, int Hkv, int Lmax, int d, float scale, int split_len,
+                    void* workspace, size_t workspace_bytes, void* stream);
+
+FA_EXPORT size_t fa_decode_workspace_size(int B, int Hq, int Lmax, int d, int split_len);
+
+/* Waits for `stream`, then returns FA_ERR_TIMEOUT if any kernel of this library recorded a
+ * device-side timeout since the previous call (and clears the record), FA_ERR_CUDA if the
+ * stream reports an error, else FA_OK. */
+FA_EXPORT fa_status fa_last_device_error(void* stream);
+
+/* Static description of a status code. */
+FA_EXPORT const char* fa_status_string(fa_status s);
+
+/* Number of streaming multiprocessors of the current device (0 on failure); the forward
+ * kernel's persistent grid uses one CTA per SM. */
+FA_EXPORT int fa_device_sm_count(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* FA_H */

@@ -1,0 +1,110 @@
+"""CPU-side checks of the C-ABI library: it builds, loads without a GPU, exports every
+function include/fa.h declares, and rejects bad arguments before touching the device."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from exact_io_aware_97_b200 import binding as fa
+from exact_io_aware_97_b200 import build as fa_build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    fa_build.build()
+    return fa.load()
+
+
+def _declared():
+    src = open(os.path.join(ROOT, "include", "fa.h")).read()
+    return sorted(set(re.findall(r"FA_EXPORT\s+[\w\s\*]+?\b(fa_\w+)\s*\(", src)))
+
+
+def test_header_declares_the_binding_names():
+    assert _declared() == sorted(fa.EXPORTED)
+
+
+def test_library_exports_every_declared_symbol(lib):
+    for name in _declared():
+        assert hasattr(lib, name), name
+    # nothing else leaks out of the library under an fa_ name
+    import subprocess
+    out = subprocess.run(["nm", "-D", "--defined-only", fa.LIB_PATH], capture_output=True, text=True).stdout
+    exported = sorted(set(re.findall(r" T (fa_\w+)", out)))
+    assert exported == _declared()
+
+
+def test_status_strings(lib):
+    for s in range(6):
+        assert fa.status_string(s)
+    assert fa.status_string(99) == "unknown status"
+
+
+def test_workspace_sizes(lib):
+    assert fa.fa_fwd_workspace_size(2, 12, 12, 2048, 2048, 64, fa.FA_BF16, False) == 0
+    n = fa.fa_fwd_workspace_size(1, 1, 1, 128, 128, 64, fa.FA_F32, False)
+    assert n >= 3 * 128 * 64 * 2
+    ws = fa.fa_decode_workspace_size(8, 64, 32768, 128, 1024)
+    assert ws >= 8 * 64 * 32 * (128 + 2) * 4
+    assert fa.fa_decode_workspace_size(0, 64, 32768, 128, 1024) == 0
+
+
+def _fwd_status(lib, **kw):
+    args = dict(q=256, k=256, v=256, o=256, lse=None, B=1, Hq=2, Hkv=1, Nq=8, Nk=8, d=64, scale=0.125, causal=1,
+                cu=None, dt=0, ws=None, wsb=0, st=None)
+    args.update(kw)
+    return lib.fa_fwd(args["q"], args["k"], args["v"], args["o"], args["lse"], args["B"], args["Hq"], args["Hkv"],
+                      args["Nq"], args["Nk"], args["d"], ctypes.c_float(args["scale"]), args["causal"], args["cu"],
+                      args["dt"], args["ws"], args["wsb"], args["st"])
+
+
+def test_fwd_rejects_before_launch(lib):
+    assert _fwd_status(lib, q=None) == fa.FA_ERR_INVALID_ARG
+    assert _fwd_status(lib, k=258) == fa.FA_ERR_INVALID_ARG          # misaligned
+    assert _fwd_status(lib, d=96) == fa.FA_ERR_UNSUPPORTED
+    assert _fwd_status(lib, Hq=3, Hkv=2) == fa.FA_ERR_UNSUPPORTED
+    assert _fwd_status(lib, scale=0.0) == fa.FA_ERR_INVALID_ARG
+    assert _fwd_status(lib, scale=float("nan")) == fa.FA_ERR_INVALID_ARG
+    assert _fwd_status(lib, B=-1) == fa.FA_ERR_INVALID_ARG
+    assert _fwd_status(lib, cu=512, Nq=8, Nk=9) == fa.FA_ERR_INVALID_ARG   # varlen needs Nq == Nk
+    assert _fwd_status(lib, cu=512, dt=1) == fa.FA_ERR_UNSUPPORTED         # fp32 varlen
+    assert _fwd_status(lib, cu=514) == fa.FA_ERR_INVALID_ARG               # misaligned offsets
+    assert _fwd_status(lib, dt=1) == fa.FA_ERR_WORKSPACE                   # fp32 needs workspace
+    assert _fwd_status(lib, dt=7) == fa.FA_ERR_INVALID_ARG
+
+
+def _dec_status(lib, **kw):
+    args = dict(q=256, kc=256, vc=256, sl=None, o=256, lse=None, B=2, Hq=8, Hkv=2, L=128, d=128, scale=0.1,
+                split=64, ws=256, wsb=1 << 30, st=None)
+    args.update(kw)
+    return lib.fa_decode(args["q"], args["kc"], args["vc"], args["sl"], args["o"], args["lse"], args["B"],
+                         args["Hq"], args["Hkv"], args["L"], args["d"], ctypes.c_float(args["scale"]),
+                         args["split"], args["ws"], args["wsb"], args["st"])
+
+
+def test_decode_rejects_before_launch(lib):
+    assert _dec_status(lib, o=None) == fa.FA_ERR_INVALID_ARG
+    assert _dec_status(lib, vc=264) == fa.FA_ERR_INVALID_ARG
+    assert _dec_status(lib, Hq=48, Hkv=2) == fa.FA_ERR_UNSUPPORTED   # group of 24 > 16
+    assert _dec_status(lib, split=100) == fa.FA_ERR_UNSUPPORTED      # not a multiple of 64
+    assert _dec_status(lib, d=80) == fa.FA_ERR_UNSUPPORTED
+    assert _dec_status(lib, ws=None) == fa.FA_ERR_WORKSPACE
+    assert _dec_status(lib, wsb=16) == fa.FA_ERR_WORKSPACE
+    assert _dec_status(lib, L=0) == fa.FA_ERR_INVALID_ARG
+    assert _dec_status(lib, sl=258) == fa.FA_ERR_INVALID_ARG
+
+
+def test_empty_problems_are_noops(lib):
+    # B == 0 or Nq == 0: valid, nothing launched
+    assert _fwd_status(lib, B=0) == fa.FA_OK
+    assert _fwd_status(lib, Nq=0) == fa.FA_OK
+    assert _dec_status(lib, B=0) == fa.FA_OK
+
+
+def test_binding_raises_fa_error(lib):
+    with pytest.raises(fa.FaError) as e:
+        fa.fa_fwd(256, 256, 256, 256, None, 1, 2, 1, 8, 8, 96, 0.1, 1, stream=0)
+    assert e.value.status == fa.FA_ERR_UNSUPPORTED

@@ -1,0 +1,186 @@
+"""GPU parity of fa_fwd (through the C ABI) against the fp64 oracle on the same inputs."""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle as oracle_mod
+import synth_inputs as si
+from exact_io_aware_97_b200 import binding as fa
+from parity import check_lse, check_out, dev_bf16, dev_f32, host64
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def orc():
+    return oracle_mod.get()
+
+
+def _inputs(seed, B, Nq, Nk, Hq, Hkv, d, dtype="bf16"):
+    q = si.normal(seed, si.Q, (B, Nq, Hq, d), dtype)
+    k = si.normal(seed, si.K, (B, Nk, Hkv, d), dtype)
+    v = si.normal(seed, si.V, (B, Nk, Hkv, d), dtype)
+    return q, k, v
+
+
+def _run_fixed(q, k, v, causal, scale):
+    o, lse = fa.forward(dev_bf16(q), dev_bf16(k), dev_bf16(v), causal=causal, scale=scale)
+    torch.cuda.synchronize()
+    assert fa.fa_last_device_error() == fa.FA_OK
+    return host64(o), host64(lse)
+
+
+SMALL = [
+    # B, Nq, Nk, Hq, Hkv, d, causal
+    (1, 1, 1, 1, 1, 64, 0),
+    (1, 17, 17, 2, 1, 64, 1),
+    (2, 127, 127, 4, 2, 128, 1),
+    (1, 129, 129, 2, 2, 128, 0),
+    (1, 255, 300, 4, 1, 64, 1),
+    (2, 257, 257, 8, 2, 128, 1),
+    (1, 300, 200, 2, 1, 128, 1),   # Nq > Nk causal: the first 100 rows see no key
+    (1, 640, 640, 2, 2, 64, 1),
+    (3, 513, 513, 6, 3, 128, 0),
+    (1, 1000, 1000, 16, 2, 128, 1),
+    (2, 384, 1500, 4, 4, 64, 0),
+    (1, 200, 1029, 8, 1, 128, 1),  # Nq < Nk causal: bottom-right aligned window
+]
+
+
+@pytest.mark.parametrize("shape", SMALL, ids=[str(s) for s in SMALL])
+def test_fwd_small_shapes(orc, shape):
+    B, Nq, Nk, Hq, Hkv, d, causal = shape
+    q, k, v = _inputs(7000 + Nq + Nk + d, B, Nq, Nk, Hq, Hkv, d)
+    scale = 1.0 / math.sqrt(d)
+    o, lse = _run_fixed(q, k, v, causal, scale)
+    o_ref, lse_ref = orc.attention(q, k, v, scale, causal=bool(causal))
+    check_out(o, o_ref)
+    check_lse(lse, lse_ref)
+
+
+def test_fwd_single_head_f32_inputs(orc):
+    """fp32 Q/K/V [1,128,1,64], non-causal, scale 1/8: inputs rounded to bf16 on the device,
+    fp32 output; compared with the oracle fed the same rounded values."""
+    w = si.WORKLOADS["single_head_f32"]
+    q, k, v = _inputs(w["seed"], 1, 128, 128, 1, 1, 64, dtype="f32")
+    o, lse = fa.forward(dev_f32(q), dev_f32(k), dev_f32(v), causal=False, scale=0.125)
+    torch.cuda.synchronize()
+    assert o.dtype == torch.float32
+    rq, rk, rv = (si.round_bf16(x) for x in (q, k, v))
+    o_ref, lse_ref = orc.attention(rq, rk, rv, 0.125)
+    check_out(host64(o), o_ref, bf16_out=False)
+    check_lse(host64(lse), lse_ref)
+    # information only: distance to the unrounded fp32 problem
+    o_raw, _ = orc.attention(q, k, v, 0.125)
+    assert np.abs(host64(o) - o_raw).max() < 0.05
+
+
+@pytest.mark.parametrize("seed_off", [0, 10000, 20000])
+def test_fwd_mha_causal_2k_full(orc, seed_off):
+    """B=2, H=12, N=2048, d=64, causal, bf16: every output element against the oracle."""
+    w = si.WORKLOADS["mha_causal_2k"]
+    q, k, v = _inputs(w["seed"] + seed_off, w["B"], w["N"], w["N"], w["Hq"], w["Hkv"], w["d"])
+    scale = 1.0 / math.sqrt(w["d"])
+    o, lse = _run_fixed(q, k, v, True, scale)
+    o_ref, lse_ref = orc.attention(q, k, v, scale, causal=True)
+    check_out(o, o_ref)
+    check_lse(lse, lse_ref)
+
+
+def _sample_rows(seed, B, Hq, nq_of_b, n_random):
+    """(b, h, i) rows: the first and last 128 rows of a few heads plus random rows."""
+    rows = []
+    u = si.uniform_ints(seed, 11, 3 * n_random, 0, 1 << 30)
+    for t in range(n_random):
+        b = int(u[3 * t] % B)
+        nq = nq_of_b(b)
+        if nq == 0:
+            continue
+        rows.append((b, int(u[3 * t + 1] % Hq), int(u[3 * t + 2] % nq)))
+    for b in range(B):
+        nq = nq_of_b(b)
+        for h in (0, Hq - 1):
+            for i in list(range(min(128, nq))) + list(range(max(0, nq - 128), nq)):
+                rows.append((b, h, i))
+    return np.array(sorted(set(rows)), dtype=np.int64)
+
+
+def test_fwd_gqa_causal_8k_sampled(orc):
+    """B=1, Hq=64, Hkv=8, N=8192, d=128, causal (the benchmark workload, same launch):
+    sampled rows against the oracle, plus bitwise repeatability."""
+    w = si.WORKLOADS["gqa_causal_8k"]
+    B, N, Hq, Hkv, d = w["B"], w["N"], w["Hq"], w["Hkv"], w["d"]
+    q, k, v = _inputs(w["seed"], B, N, N, Hq, Hkv, d)
+    scale = 1.0 / math.sqrt(d)
+    qd, kd, vd = dev_bf16(q), dev_bf16(k), dev_bf16(v)
+    o1, l1 = fa.forward(qd, kd, vd, causal=True, scale=scale)
+    o2, l2 = fa.forward(qd, kd, vd, causal=True, scale=scale)
+    torch.cuda.synchronize()
+    assert torch.equal(o1, o2) and torch.equal(l1, l2)
+    rows = _sample_rows(w["seed"], B, Hq, lambda b: N, 4096)
+    o_ref, lse_ref = orc.attention_rows(q, k, v, scale, rows, causal=True)
+    o = host64(o1)
+    lse = host64(l1)
+    check_out(o[rows[:, 0], rows[:, 2], rows[:, 1]], o_ref)
+    check_lse(lse[rows[:, 0], rows[:, 1], rows[:, 2]], lse_ref)
+
+
+def _varlen_inputs(seed, lengths, Hq, Hkv, d):
+    cu = si.cu_seqlens(lengths)
+    T = int(cu[-1])
+    q = si.normal(seed, si.Q, (T, Hq, d))
+    k = si.normal(seed, si.K, (T, Hkv, d))
+    v = si.normal(seed, si.V, (T, Hkv, d))
+    return cu, q, k, v
+
+
+@pytest.mark.parametrize("lengths,Hq,Hkv,d", [
+    ([1, 130, 256, 257, 511, 3], 4, 2, 128),
+    ([600, 0, 17, 1024, 255], 8, 2, 64),
+    ([5000], 2, 1, 128),
+])
+def test_fwd_varlen_small(orc, lengths, Hq, Hkv, d):
+    cu, q, k, v = _varlen_inputs(8000 + sum(lengths), lengths, Hq, Hkv, d)
+    scale = 1.0 / math.sqrt(d)
+    cud = torch.from_numpy(cu).cuda()
+    o, lse = fa.forward(dev_bf16(q), dev_bf16(k), dev_bf16(v), causal=True, scale=scale, cu_seqlens=cud)
+    torch.cuda.synchronize()
+    o_ref, lse_ref = orc.attention(q, k, v, scale, causal=True, cu_seqlens=cu)
+    check_out(host64(o), o_ref)
+    check_lse(host64(lse), lse_ref)
+
+
+def test_fwd_varlen_gqa_causal_sampled(orc):
+    """16 sequences, lengths U[256, 8192] from the seed, Hq=32, Hkv=8, d=128, causal, packed."""
+    w = si.WORKLOADS["varlen_gqa_causal"]
+    lengths = si.varlen_lengths(w["seed"], w["nseq"], w["len_lo"], w["len_hi"])
+    cu, q, k, v = _varlen_inputs(w["seed"], lengths, w["Hq"], w["Hkv"], w["d"])
+    scale = 1.0 / math.sqrt(w["d"])
+    cud = torch.from_numpy(cu).cuda()
+    o, lse = fa.forward(dev_bf16(q), dev_bf16(k), dev_bf16(v), causal=True, scale=scale, cu_seqlens=cud)
+    torch.cuda.synchronize()
+    rows = _sample_rows(w["seed"], len(lengths), w["Hq"], lambda b: int(lengths[b]), 4096)
+    o_ref, lse_ref = orc.attention_rows(q, k, v, scale, rows, causal=True, cu_seqlens=cu)
+    tok = cu[rows[:, 0]] + rows[:, 2]
+    check_out(host64(o)[tok, rows[:, 1]], o_ref)
+    check_lse(host64(lse)[rows[:, 1], tok], lse_ref)
+
+
+def test_fwd_lse_optional_and_noncausal_gqa(orc):
+    B, N, Hq, Hkv, d = 2, 700, 8, 2, 128
+    q, k, v = _inputs(9100, B, N, N, Hq, Hkv, d)
+    qd, kd, vd = dev_bf16(q), dev_bf16(k), dev_bf16(v)
+    o = torch.empty_like(qd)
+    fa.fa_fwd(qd, kd, vd, o, None, B, Hq, Hkv, N, N, d, 0.1, 0)
+    torch.cuda.synchronize()
+    o_ref, _ = orc.attention(q, k, v, 0.1)
+    check_out(host64(o), o_ref)
+
+
+def test_fwd_rejects_without_launch():
+    qd = torch.zeros(1, 16, 2, 96, dtype=torch.bfloat16, device="cuda")
+    with pytest.raises(fa.FaError) as e:
+        fa.forward(qd, qd, qd)
+    assert e.value.status == fa.FA_ERR_UNSUPPORTED
