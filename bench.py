@@ -96,6 +96,28 @@ def ncu_traffic(key: str):
     return e.get("bytes_per_launch")
 
 
+# ----------------------------------------------------------------------------- ranks
+def replica_seed(base_seed: int, rank: int) -> int:
+    """Each rank runs its own replica of the workload on its own seeded inputs."""
+    return base_seed + 100000 * rank
+
+
+def max_over_ranks(x: float, device=None) -> float:
+    """Max of a per-rank time over the process group (identity without one)."""
+    import torch
+    import torch.distributed as dist
+    if not dist.is_available() or not dist.is_initialized() or dist.get_world_size() == 1:
+        return x
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def aggregate_rate(units_per_replica: float, world: int, max_ms: float) -> float:
+    """Whole-job rate: the units all ranks processed over the slowest rank's time (per second)."""
+    return world * units_per_replica / (max_ms * 1e-3)
+
+
 # ----------------------------------------------------------------------------- clocks
 class ClockSampler:
     FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
@@ -187,13 +209,6 @@ def run_device(args):
             dist.barrier()
         torch.cuda.synchronize()
 
-    def max_over_ranks(x: float) -> float:
-        if world == 1:
-            return x
-        t = torch.tensor([x], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
-
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
 
     def l2_flush():
@@ -202,10 +217,10 @@ def run_device(args):
     # ---- inputs (each rank its own replica, seeded by the workload seed + rank)
     w = FWD
     B, N, Hq, Hkv, d = w["B"], w["N"], w["Hq"], w["Hkv"], w["d"]
-    seed = w["seed"] + 100000 * rank
-    h_q = torch.from_numpy(si.normal(seed, si.Q, (B, N, Hq, d))).to(torch.bfloat16).pin_memory()
-    h_k = torch.from_numpy(si.normal(seed, si.K, (B, N, Hkv, d))).to(torch.bfloat16).pin_memory()
-    h_v = torch.from_numpy(si.normal(seed, si.V, (B, N, Hkv, d))).to(torch.bfloat16).pin_memory()
+    seed = replica_seed(w["seed"], rank)
+    h_q = torch.from_numpy(inputs("fwd", seed, si.Q, (B, N, Hq, d))).to(torch.bfloat16).pin_memory()
+    h_k = torch.from_numpy(inputs("fwd", seed, si.K, (B, N, Hkv, d))).to(torch.bfloat16).pin_memory()
+    h_v = torch.from_numpy(inputs("fwd", seed, si.V, (B, N, Hkv, d))).to(torch.bfloat16).pin_memory()
     q, k, v = h_q.to(dev), h_k.to(dev), h_v.to(dev)
     o = torch.empty_like(q)
     lse = torch.empty((B, Hq, N), dtype=torch.float32, device=dev)
@@ -213,12 +228,19 @@ def run_device(args):
     h_lse = torch.empty(lse.shape, dtype=torch.float32).pin_memory()
     scale = 1.0 / math.sqrt(d)
 
+    do_fwd = args.only in ("all", "fwd")
+    do_dec = args.only in ("all", "dec")
+    if not do_fwd:
+        del q, k, v, o, lse
     wd = DEC
-    dseed = wd["seed"] + 100000 * rank
+    dseed = replica_seed(wd["seed"], rank)
     dB, dHq, dHkv, L, dd, split = wd["B"], wd["Hq"], wd["Hkv"], wd["L"], wd["d"], wd["split"]
-    h_dq = torch.from_numpy(si.normal(dseed, si.Q, (dB, dHq, dd))).to(torch.bfloat16).pin_memory()
-    h_kc = torch.from_numpy(si.normal(dseed, si.KCACHE, (dB, L, dHkv, dd))).to(torch.bfloat16).pin_memory()
-    h_vc = torch.from_numpy(si.normal(dseed, si.VCACHE, (dB, L, dHkv, dd))).to(torch.bfloat16).pin_memory()
+    if not do_dec:
+        dB = 1  # a token-sized decode problem keeps the code below uniform
+        dq = kc = vc = None
+    h_dq = torch.from_numpy(inputs("dec", dseed, si.Q, (dB, dHq, dd))).to(torch.bfloat16).pin_memory()
+    h_kc = torch.from_numpy(inputs("dec", dseed, si.KCACHE, (dB, L, dHkv, dd))).to(torch.bfloat16).pin_memory()
+    h_vc = torch.from_numpy(inputs("dec", dseed, si.VCACHE, (dB, L, dHkv, dd))).to(torch.bfloat16).pin_memory()
     dq, kc, vc = h_dq.to(dev), h_kc.to(dev), h_vc.to(dev)
     do = torch.empty((dB, dHq, dd), dtype=torch.bfloat16, device=dev)
     dlse = torch.empty((dB, dHq), dtype=torch.float32, device=dev)
@@ -255,8 +277,8 @@ def run_device(args):
         ms = [a.elapsed_time(b) for a, b in evs]
         return ms
 
-    fwd_ms = timed_launches(call_fwd, args.steps, args.warmup)
-    dec_ms = timed_launches(call_dec, args.steps, args.warmup)
+    fwd_ms = timed_launches(call_fwd, args.steps, args.warmup) if do_fwd else [float("nan")]
+    dec_ms = timed_launches(call_dec, args.steps, args.warmup) if do_dec else [float("nan")]
     if fa.fa_last_device_error(st) != fa.FA_OK:
         raise RuntimeError("device-side timeout recorded during the benchmark")
 
@@ -291,16 +313,16 @@ def run_device(args):
         h_do.copy_(do, non_blocking=True)
 
     e2e_steps = max(3, args.steps // 4)
-    fwd_e2e_ms = e2e(e2e_steps, 1, fwd_e2e_body)
-    dec_e2e_ms = e2e(e2e_steps, 1, dec_e2e_body)
+    fwd_e2e_ms = e2e(e2e_steps, 1, fwd_e2e_body) if (do_fwd and not args.no_e2e) else float("nan")
+    dec_e2e_ms = e2e(e2e_steps, 1, dec_e2e_body) if (do_dec and not args.no_e2e) else float("nan")
     torch.cuda.synchronize()
     clocks.stop()
 
     # ---- reduce over ranks (max time)
-    fwd_mean = max_over_ranks(sum(fwd_ms) / len(fwd_ms))
-    dec_mean = max_over_ranks(sum(dec_ms) / len(dec_ms))
-    fwd_e2e_ms = max_over_ranks(fwd_e2e_ms)
-    dec_e2e_ms = max_over_ranks(dec_e2e_ms)
+    fwd_mean = max_over_ranks(sum(fwd_ms) / len(fwd_ms), dev)
+    dec_mean = max_over_ranks(sum(dec_ms) / len(dec_ms), dev)
+    fwd_e2e_ms = max_over_ranks(fwd_e2e_ms, dev)
+    dec_e2e_ms = max_over_ranks(dec_e2e_ms, dev)
     if world > 1:
         dist.barrier()
         dist.destroy_process_group()
@@ -308,9 +330,9 @@ def run_device(args):
         return
 
     F = fwd_flops()
-    tflops = world * F / (fwd_mean * 1e-3) / 1e12
+    tflops = aggregate_rate(F, world, fwd_mean) / 1e12
     kv = dec_kv_bytes()
-    gbs = world * kv / (dec_mean * 1e-3) / 1e9
+    gbs = aggregate_rate(kv, world, dec_mean) / 1e9
     h2d_fwd = h_q.numel() * 2 + h_k.numel() * 2 + h_v.numel() * 2
     d2h_fwd = h_o.numel() * 2 + h_lse.numel() * 4
     h2d_dec = h_dq.numel() * 2 + h_kc.numel() * 2 + h_vc.numel() * 2
@@ -369,13 +391,24 @@ def run_device(args):
 
 
 # ----------------------------------------------------------------------------- CPU oracle
+_INPUTS = {}
+
+
+def inputs(key, seed, tid, shape):
+    """Seeded host inputs (float32 holding bf16 values), generated once per process."""
+    k = (key, seed, tid, tuple(shape))
+    if k not in _INPUTS:
+        _INPUTS[k] = si.normal(seed, tid, shape)
+    return _INPUTS[k]
+
+
 def _oracle_rows_fwd(orc, rows_target, threads, seed):
     """Time the oracle on `rows_target` random rows of the forward workload."""
     w = FWD
     B, N, Hq, Hkv, d = w["B"], w["N"], w["Hq"], w["Hkv"], w["d"]
-    q = si.normal(seed, si.Q, (B, N, Hq, d))
-    k = si.normal(seed, si.K, (B, N, Hkv, d))
-    v = si.normal(seed, si.V, (B, N, Hkv, d))
+    q = inputs("fwd", seed, si.Q, (B, N, Hq, d))
+    k = inputs("fwd", seed, si.K, (B, N, Hkv, d))
+    v = inputs("fwd", seed, si.V, (B, N, Hkv, d))
     u = si.uniform_ints(seed, 13, 2 * rows_target, 0, (1 << 30))
     rows = np.stack([np.zeros(rows_target, np.int64), u[0::2] % Hq, u[1::2] % N], 1)
     t = time.perf_counter()
@@ -402,9 +435,9 @@ def _oracle_dec(orc, pairs, threads, seed):
     B, Hq, Hkv, L, d = w["B"], w["Hq"], w["Hkv"], w["L"], w["d"]
     G = Hq // Hkv
     # the first `pairs` (sequence, kv-head) groups: each group's G query heads read its K/V once
-    q = si.normal(seed, si.Q, (B, Hq, d))
-    kc = si.normal(seed, si.KCACHE, (B, L, Hkv, d))
-    vc = si.normal(seed, si.VCACHE, (B, L, Hkv, d))
+    q = inputs("dec", seed, si.Q, (B, Hq, d))
+    kc = inputs("dec", seed, si.KCACHE, (B, L, Hkv, d))
+    vc = inputs("dec", seed, si.VCACHE, (B, L, Hkv, d))
     rows = []
     for p in range(pairs):
         b, g = p // Hkv, p % Hkv
@@ -469,6 +502,8 @@ def main():
     ap.add_argument("--impl", default="b200", choices=["b200", "reference"])
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--no-cpu", action="store_true", help="skip the CPU oracle baseline")
+    ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer end-to-end phases")
+    ap.add_argument("--only", default="all", choices=["all", "fwd", "dec"], help="profiling: run one kernel family")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3

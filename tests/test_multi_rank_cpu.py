@@ -1,0 +1,55 @@
+"""Multi-rank host logic of the benchmark on CPU (gloo, world size 2): replicas get distinct
+seeded inputs, per-rank times reduce to their max, and the whole-job rate counts every
+rank's units over the slowest rank's time.  No data-path collective exists to test: the
+units are independent."""
+import os
+import socket
+
+import pytest
+import torch
+import torch.distributed as dist
+import torch.multiprocessing as mp
+
+import bench
+import synth_inputs as si
+
+
+def _free_port():
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _worker(rank, world, port, out):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank), WORLD_SIZE=str(world))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        t = bench.max_over_ranks(1.5 + rank)
+        seed = bench.replica_seed(1003, rank)
+        x = torch.from_numpy(si.normal(seed, si.Q, (64,)))
+        gathered = [torch.empty_like(x) for _ in range(world)]
+        dist.all_gather(gathered, x)
+        out[rank] = (t, bool(torch.equal(gathered[0], gathered[1])))
+        dist.barrier()
+    finally:
+        dist.destroy_process_group()
+
+
+def test_two_ranks_max_time_and_distinct_replicas():
+    world = 2
+    port = _free_port()
+    with mp.Manager() as m:
+        out = m.dict()
+        mp.spawn(_worker, args=(world, port, out), nprocs=world, join=True)
+        res = dict(out)
+    assert res[0][0] == res[1][0] == 2.5
+    assert res[0][1] is False  # the two replicas' inputs differ
+
+
+def test_aggregate_rate_counts_all_ranks():
+    assert bench.aggregate_rate(1e12, 4, 1000.0) == pytest.approx(4e12)
+    assert bench.aggregate_rate(2.0, 1, 2.0) == pytest.approx(1000.0)
+
+
+def test_single_process_max_is_identity():
+    assert bench.max_over_ranks(3.25) == 3.25
