@@ -17,8 +17,9 @@ LIB_PATH = os.path.join(PKG, "libfa.so")
 FA_OK, FA_ERR_INVALID_ARG, FA_ERR_UNSUPPORTED, FA_ERR_WORKSPACE, FA_ERR_CUDA, FA_ERR_TIMEOUT = range(6)
 FA_BF16, FA_F32 = 0, 1
 
-EXPORTED = ("fa_fwd", "fa_fwd_workspace_size", "fa_decode", "fa_decode_workspace_size",
+EXPORTED = ("fa_fwd", "fa_fwd_workspace_size", "fa_decode", "fa_decode_workspace_size", "fa_decode_noalloc",
             "fa_last_device_error", "fa_status_string", "fa_device_sm_count")
+FA_DECODE_NOALLOC_SCRATCH_BYTES = 16 << 20
 
 
 class FaError(RuntimeError):
@@ -45,6 +46,8 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
     L.fa_fwd_workspace_size.restype = sz
     L.fa_decode.argtypes = [vp, vp, vp, vp, vp, vp, i, i, i, i, i, f, i, vp, sz, vp]
     L.fa_decode.restype = i
+    L.fa_decode_noalloc.argtypes = [vp, vp, vp, vp, vp, vp, i, i, i, i, i, f, i, vp]
+    L.fa_decode_noalloc.restype = i
     L.fa_decode_workspace_size.argtypes = [i, i, i, i, i]
     L.fa_decode_workspace_size.restype = sz
     L.fa_last_device_error.argtypes = [vp]
@@ -102,6 +105,17 @@ def fa_decode(q, kcache, vcache, seqlens, o, lse, B, Hq, Hkv, Lmax, d, scale, sp
                           int(Hkv), int(Lmax), int(d), float(scale), int(split_len), _ptr(workspace),
                           int(workspace_bytes), _stream(stream))
     _check(st, "fa_decode")
+
+
+def fa_decode_noalloc(q, kcache, vcache, seqlens, o, lse, B, Hq, Hkv, Lmax, d, scale, split_len,
+                      stream=None) -> None:
+    """fa_decode with its scratch in the library's static device array (no allocation).
+    For callers that cannot allocate device memory; calls that overlap on the GPU race, and
+    the first call on a device should come before any stream capture (see include/fa.h)."""
+    st = load().fa_decode_noalloc(_ptr(q), _ptr(kcache), _ptr(vcache), _ptr(seqlens), _ptr(o), _ptr(lse), int(B),
+                                  int(Hq), int(Hkv), int(Lmax), int(d), float(scale), int(split_len),
+                                  _stream(stream))
+    _check(st, "fa_decode_noalloc")
 
 
 def fa_decode_workspace_size(B, Hq, Lmax, d, split_len) -> int:

@@ -273,3 +273,50 @@ fa_status fa_last_device_error(void* stream) {
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------------------
+// fa_decode_noalloc: fa_decode with its scratch in a static device array, for callers that
+// cannot allocate device memory (see include/fa.h).
+namespace fa {
+namespace {
+
+// The split partials of fa_decode_noalloc.  In host code this name is only a stand-in for
+// the symbol; its device address comes from cudaGetSymbolAddress (per device).
+static __device__ __align__(256) unsigned char g_decode_noalloc_scratch[FA_DECODE_NOALLOC_SCRATCH_BYTES];
+
+std::mutex g_noalloc_mu;
+void* g_noalloc_ptr[64] = {};
+
+// Device address of the scratch array on the current device, looked up once per device.
+fa_status noalloc_scratch(void** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return FA_ERR_CUDA;
+  std::lock_guard<std::mutex> lock(g_noalloc_mu);
+  if (g_noalloc_ptr[dev] == nullptr) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_decode_noalloc_scratch) != cudaSuccess || p == nullptr) return FA_ERR_CUDA;
+    g_noalloc_ptr[dev] = p;
+  }
+  *out = g_noalloc_ptr[dev];
+  return FA_OK;
+}
+
+}  // namespace
+}  // namespace fa
+
+extern "C" fa_status fa_decode_noalloc(const void* q, const void* kcache, const void* vcache, const int32_t* seqlens,
+                                       void* o, float* lse, int B, int Hq, int Hkv, int Lmax, int d, float scale,
+                                       int split_len, void* stream) {
+  // Argument checks of fa_decode, without a workspace: a valid non-empty problem stops at the
+  // workspace check (nothing launched); anything else is returned as is.
+  const fa_status pre = fa_decode(q, kcache, vcache, seqlens, o, lse, B, Hq, Hkv, Lmax, d, scale, split_len,
+                                  nullptr, 0, stream);
+  if (pre != FA_ERR_WORKSPACE) return pre;
+  if (fa_decode_workspace_size(B, Hq, Lmax, d, split_len) > (size_t)FA_DECODE_NOALLOC_SCRATCH_BYTES)
+    return FA_ERR_WORKSPACE;
+  void* scratch = nullptr;
+  const fa_status st = fa::noalloc_scratch(&scratch);
+  if (st != FA_OK) return st;
+  return fa_decode(q, kcache, vcache, seqlens, o, lse, B, Hq, Hkv, Lmax, d, scale, split_len, scratch,
+                   (size_t)FA_DECODE_NOALLOC_SCRATCH_BYTES, stream);
+}

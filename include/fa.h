@@ -98,6 +98,34 @@ FA_EXPORT fa_status fa_decode(const void* q, const void* kcache, const void* vca
 
 FA_EXPORT size_t fa_decode_workspace_size(int B, int Hq, int Lmax, int d, int split_len);
 
+/* Largest scratch, in bytes, that fa_decode_noalloc can use (16 MiB). */
+#define FA_DECODE_NOALLOC_SCRATCH_BYTES (16u << 20)
+
+/* fa_decode for callers that cannot allocate device memory.
+ *
+ * Some callers have no way to call cudaMalloc on this path: a host program that only
+ * receives its input and output buffers from someone else (a plugin inside another
+ * framework's memory pool), or a latency-critical loop where an allocation, which can
+ * synchronise the device, is not allowed.  This entry point takes the same arguments as
+ * fa_decode minus the workspace and allocates nothing.  The pages describe no such entry
+ * point; it exists only for these callers.
+ *
+ * Scratch: the split partials live in one static device array of
+ * FA_DECODE_NOALLOC_SCRATCH_BYTES in this library, which every GPU that loads the library
+ * holds until the process exits.  Problems whose scratch need (fa_decode_workspace_size)
+ * exceeds it are rejected with FA_ERR_WORKSPACE before anything is launched; the decode
+ * workload B=8, Hq=64, d=128, cache 32768, splits of 1024 needs about 8.7 MB.
+ * No part of the scratch has to start at zero: every partial the merge reads is written by
+ * the same call.  All calls share the array, so calls that overlap on the GPU (on
+ * different streams, or on one stream from different threads without ordering) race and
+ * give wrong results; order them on one stream.
+ * The first call on each device looks up the array's device address (with that device
+ * current) and caches it; make that first call before any stream capture.
+ * Other arguments, results and errors are those of fa_decode. */
+FA_EXPORT fa_status fa_decode_noalloc(const void* q, const void* kcache, const void* vcache, const int32_t* seqlens,
+                                      void* o, float* lse, int B, int Hq, int Hkv, int Lmax, int d, float scale,
+                                      int split_len, void* stream);
+
 /* Waits for `stream`, then returns FA_ERR_TIMEOUT if any kernel of this library recorded a
  * device-side timeout since the previous call (and clears the record), FA_ERR_CUDA if the
  * stream reports an error, else FA_OK. */
