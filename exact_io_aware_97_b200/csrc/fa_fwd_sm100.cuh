@@ -8,11 +8,13 @@
 // the output accumulator is rescaled by the same factor and P V is added to it.  Only O
 // and the per-row logsumexp are written to device memory.
 //
-// B200 mapping (one persistent CTA per SM, 320 threads):
-//   warps 0-3  softmax for query tile 0 (thread = row), then its epilogue
-//   warps 4-7  softmax for query tile 1
-//   warp  8    tcgen05.mma issuer (one thread) and TMEM owner
-//   warp  9    TMA producer (one thread)
+// B200 mapping (one persistent CTA per SM, 384 threads):
+//   warps 0-3   softmax for query tile 0 (thread = row), then its epilogue
+//   warps 4-7   softmax for query tile 1
+//   warp  8     tcgen05.mma issuer and TMEM owner
+//   warp  9     TMA producer
+//   warps 10-11 idle (they complete the control warpgroup for the register split)
+// The issuing warps run converged and let one elected lane issue each instruction.
 // A work unit is 256 query rows (two 128-row tiles) of one (sequence, query head).  Units
 // are ordered longest-first (causal cost grows with the query tile index) and dealt to
 // CTAs in a snake order.  K and V tiles (128 keys each) flow through a shared-memory ring
@@ -44,10 +46,21 @@ struct FwdParams {
 constexpr int kBM = 128;        // query rows per tile
 constexpr int kBN = 128;        // keys per K/V tile
 constexpr int kUnitRows = 256;  // two query tiles per work unit
-constexpr int kFwdThreads = 320;
+constexpr int kFwdThreads = 384;
+// Register split by warpgroup, set with setmaxnreg after the common prologue.  The launch
+// gives 384 threads x 168 registers = 64512; softmax warpgroups take 2 x 128 x 208 and the
+// control warpgroup (MMA, TMA, two idle warps) 128 x 88, the same total (and the same per
+// SM sub-partition: two softmax warps and one control warp each).
+constexpr int kSoftmaxRegs = 208;
+constexpr int kControlRegs = 88;
 constexpr int kMaxVarlenB = 1024;
 constexpr int kMaxVarlenT = 1024;
 constexpr float kRescaleThreshold = 8.0f;
+// Column pairs (of each group of 8) whose 2^x runs on the FMA pipe in unmasked tiles, and
+// pairs packed to bf16 with integer operations instead of the conversion unit: together
+// they move work off the special-function pipe, which otherwise bounds the softmax.
+constexpr uint32_t kEmuPairMask = 0x00;
+constexpr uint32_t kIntPackPairMask = 0x00;
 
 template <int D>
 struct FwdCfg {
@@ -56,7 +69,7 @@ struct FwdCfg {
   static constexpr int kStages = (D == 128) ? 4 : 8;
   static constexpr int kQBytes = 2 * kTileBytes;
   static constexpr int kRingBytes = kStages * kTileBytes;
-  static constexpr int kNumBars = 2 + 2 * kStages + 8;
+  static constexpr int kNumBars = 2 + 2 * kStages + 10;
   static constexpr int kBarBytes = kNumBars * 8 + 16;
   static constexpr int kSchedBytes = kMaxVarlenB * 2 + kMaxVarlenT * 4 + 16;
   static constexpr int kSmemBytes = 1024 + kQBytes + kRingBytes + kBarBytes + kSchedBytes;
@@ -168,10 +181,10 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
   uint64_t* q_empty = bars + 1;
   uint64_t* full = bars + 2;
   uint64_t* empty = bars + 2 + NS;
-  uint64_t* s_full = bars + 2 + 2 * NS;  // [2]
-  uint64_t* p_full = s_full + 2;         // [2]
-  uint64_t* pv_done = p_full + 2;        // [2]
-  uint64_t* o_free = pv_done + 2;        // [2]
+  uint64_t* s_full = bars + 2 + 2 * NS;  // [tile]
+  uint64_t* p_half = s_full + 2;         // [tile][half]: P columns 0-63 / 64-127 written
+  uint64_t* pv_done = p_half + 4;        // [tile]
+  uint64_t* o_free = pv_done + 2;        // [tile]
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + C::kNumBars);
   int* sched_misc = reinterpret_cast<int*>(tmem_slot + 2);  // [0] = T, [1] = total tiles
   uint8_t* sched_mem = reinterpret_cast<uint8_t*>(bars) + C::kBarBytes;
@@ -190,7 +203,8 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(s_full + i, 1);
-      mbar_init(p_full + i, kBM);
+      mbar_init(p_half + 2 * i, kBM);
+      mbar_init(p_half + 2 * i + 1, kBM);
       mbar_init(pv_done + i, 1);
       mbar_init(o_free + i, kBM);
     }
@@ -256,9 +270,11 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
+  if (warp >= 8) {
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kControlRegs));
   if (warp == 9) {
     // ================================================================ TMA producer
-    if (lane == 0) {
+    {
       const uint64_t kv_policy = policy_evict_last();
       uint32_t g = 0, qcount = 0;
       UnitIter it;
@@ -267,23 +283,23 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       for (int u = it.next(sch.U); u >= 0 && ok; u = it.next(sch.U)) {
         Unit un;
         decode_unit(p, sch, wk, u, un);
-        if (qcount > 0 && !mbar_wait(q_empty, (qcount - 1) & 1)) break;
+        if (qcount > 0 && !warp_wait(q_empty, (qcount - 1) & 1)) break;
         const int ntile = un.valid[1] ? 2 : 1;
-        mbar_arrive_expect_tx(q_full, ntile * C::kTileBytes);
+        mbar_arrive_expect_tx_elect(q_full, ntile * C::kTileBytes);
         for (int i = 0; i < ntile; ++i)
           for (int c = 0; c < D / 64; ++c)
-            tma_load_3d(sQ + i * C::kTileBytes + c * C::kChunkBytes, &tmQ, c * 64, un.h,
+            tma_load_3d_elect(sQ + i * C::kTileBytes + c * C::kChunkBytes, &tmQ, c * 64, un.h,
                         un.q_start + un.row0 + i * kBM, q_full);
         for (int j = 0; j < un.nmax && ok; ++j) {
           for (int kv = 0; kv < 2; ++kv) {
             const uint32_t slot = g % NS;
-            if (g >= (uint32_t)NS && !mbar_wait(empty + slot, ((g / NS) - 1) & 1)) {
+            if (g >= (uint32_t)NS && !warp_wait(empty + slot, ((g / NS) - 1) & 1)) {
               ok = false;
               break;
             }
-            mbar_arrive_expect_tx(full + slot, C::kTileBytes);
+            mbar_arrive_expect_tx_elect(full + slot, C::kTileBytes);
             for (int c = 0; c < D / 64; ++c)
-              tma_load_3d_hint(sRing + slot * C::kTileBytes + c * C::kChunkBytes, kv ? &tmV : &tmK, c * 64,
+              tma_load_3d_hint_elect(sRing + slot * C::kTileBytes + c * C::kChunkBytes, kv ? &tmV : &tmK, c * 64,
                                un.kvh, un.k_start + j * kBN, full + slot, kv_policy);
             ++g;
           }
@@ -294,7 +310,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
     __syncwarp();
   } else if (warp == 8) {
     // ================================================================ MMA issuer
-    if (lane == 0) {
+    {
       constexpr uint32_t idS = idesc_bf16_f32(kBM, kBN, false);
       constexpr uint32_t idPV = idesc_bf16_f32(kBM, D, true);
       const uint32_t qbase = smem_u32(sQ);
@@ -311,39 +327,44 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
           const uint32_t off = (kk >> 2) * C::kChunkBytes + (kk & 3) * 32;
           const uint64_t a = smem_desc_sw128(qbase + i * C::kTileBytes + off, 16, 1024);
           const uint64_t bd = smem_desc_sw128(rbase + slot * C::kTileBytes + off, 16, 1024);
-          umma_ss(tmem + i * kBN, a, bd, idS, kk > 0 ? 1u : 0u);
+          umma_ss_elect(tmem + i * kBN, a, bd, idS, kk > 0 ? 1u : 0u);
         }
       };
-      auto issue_PV = [&](int i, uint32_t slot, bool acc) {
+      // O_i (+)= P_i V for the keys of one half (8 k-steps of 16 keys in all).
+      auto issue_PV_half = [&](int i, uint32_t slot, int half, bool acc) {
 #pragma unroll
-        for (int kk = 0; kk < kBN / 16; ++kk) {
+        for (int k4 = 0; k4 < kBN / 32; ++k4) {
+          const int kk = half * (kBN / 32) + k4;
           const uint64_t bd = smem_desc_sw128(rbase + slot * C::kTileBytes + kk * 16 * 128, C::kChunkBytes, 1024);
-          umma_ts(tmem + C::kColO + i * D, tmem + i * kBN + kk * 8, bd, idPV, (acc || kk > 0) ? 1u : 0u);
+          umma_ts_elect(tmem + C::kColO + i * D, tmem + i * kBN + kk * 8, bd, idPV, (acc || kk > 0) ? 1u : 0u);
         }
       };
       auto wait_full = [&](uint32_t gi) -> bool {
-        if (!mbar_wait(full + (gi % NS), (gi / NS) & 1)) return false;
+        if (!warp_wait(full + (gi % NS), (gi / NS) & 1)) return false;
         tc_fence_after();
         return true;
       };
       auto pv_step = [&](int i, int j, uint32_t vslot) -> bool {
-        if (j == 0 && ounits[i] > 0 && !mbar_wait(o_free + i, (ounits[i] - 1) & 1)) return false;
-        if (!mbar_wait(p_full + i, pcnt[i] & 1)) return false;
+        if (j == 0 && ounits[i] > 0 && !warp_wait(o_free + i, (ounits[i] - 1) & 1)) return false;
+        // the first half of P is consumed while the softmax still writes the second
+        for (int half = 0; half < 2; ++half) {
+          if (!warp_wait(p_half + 2 * i + half, pcnt[i] & 1)) return false;
+          tc_fence_after();
+          issue_PV_half(i, vslot, half, j > 0);
+        }
         ++pcnt[i];
-        tc_fence_after();
-        issue_PV(i, vslot, j > 0);
-        umma_commit(pv_done + i);
+        umma_commit_elect(pv_done + i);
         return true;
       };
 
       for (int u = it.next(sch.U); u >= 0 && ok; u = it.next(sch.U)) {
         Unit un;
         decode_unit(p, sch, wk, u, un);
-        if (!mbar_wait(q_full, qcount & 1)) break;
+        if (!warp_wait(q_full, qcount & 1)) break;
         tc_fence_after();
         const int nmax = un.nmax;
         if (nmax == 0) {
-          umma_commit(q_empty);
+          umma_commit_elect(q_empty);
           ++qcount;
           continue;
         }
@@ -352,10 +373,10 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         for (int i = 0; i < 2; ++i)
           if (un.n[i] > 0) {
             issue_S(i, g % NS);
-            umma_commit(s_full + i);
+            umma_commit_elect(s_full + i);
           }
-        umma_commit(empty + (g % NS));
-        if (nmax == 1) umma_commit(q_empty);
+        umma_commit_elect(empty + (g % NS));
+        if (nmax == 1) umma_commit_elect(q_empty);
         for (int j = 0; j < nmax && ok; ++j) {
           const uint32_t gv = g + 2 * j + 1;
           const uint32_t gk = g + 2 * j + 2;
@@ -365,18 +386,18 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
             if (!wait_full(gk)) { ok = false; break; }
             if (j + 1 < un.n[0]) {
               issue_S(0, gk % NS);
-              umma_commit(s_full + 0);
+              umma_commit_elect(s_full + 0);
             }
           }
           if (j < un.n[1] && !pv_step(1, j, gv % NS)) { ok = false; break; }
-          umma_commit(empty + (gv % NS));
+          umma_commit_elect(empty + (gv % NS));
           if (j + 1 < nmax) {
             if (j + 1 < un.n[1]) {
               issue_S(1, gk % NS);
-              umma_commit(s_full + 1);
+              umma_commit_elect(s_full + 1);
             }
-            umma_commit(empty + (gk % NS));
-            if (j + 2 == nmax) umma_commit(q_empty);
+            umma_commit_elect(empty + (gk % NS));
+            if (j + 2 == nmax) umma_commit_elect(q_empty);
           }
         }
         g += 2 * nmax;
@@ -386,7 +407,9 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       }
     }
     __syncwarp();
+  }
   } else {
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kSoftmaxRegs));
     // ================================================================ softmax + epilogue
     const int i = warp >> 2;            // query tile of this warpgroup
     const int r = threadIdx.x & 127;    // row within the tile = TMEM lane
@@ -431,56 +454,73 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
           for (int c = 0; c < 128; ++c)
             if (c >= lim) s[c] = -INFINITY;
         }
-        float mx0 = s[0], mx1 = s[1], mx2 = s[2], mx3 = s[3];
+        // row max: 16 independent chains of three-input max, then a three-level tree
+        float mx[16];
 #pragma unroll
-        for (int c = 4; c < 128; c += 4) {
-          mx0 = fmaxf(mx0, s[c]);
-          mx1 = fmaxf(mx1, s[c + 1]);
-          mx2 = fmaxf(mx2, s[c + 2]);
-          mx3 = fmaxf(mx3, s[c + 3]);
+        for (int q = 0; q < 16; ++q) {
+          mx[q] = fmax3(s[q], s[q + 16], s[q + 32]);
+          mx[q] = fmax3(mx[q], s[q + 48], s[q + 64]);
+          mx[q] = fmax3(mx[q], s[q + 80], s[q + 96]);
+          mx[q] = fmaxf(mx[q], s[q + 112]);
         }
-        const float m_tile = fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3)) * tau;
+        float my[6];
+#pragma unroll
+        for (int q = 0; q < 5; ++q) my[q] = fmax3(mx[3 * q], mx[3 * q + 1], mx[3 * q + 2]);
+        my[5] = mx[15];
+        const float m_tile = fmaxf(fmax3(my[0], my[1], my[2]), fmax3(my[3], my[4], my[5])) * tau;
         const float m_new = fmaxf(m_ref, m_tile);
         const bool need = m_new - m_ref > kRescaleThreshold;  // false when both are -inf
         const bool warp_need = __any_sync(0xffffffffu, need);
         const float alpha = need ? ex2_approx(m_ref - m_new) : 1.f;
         if (need) m_ref = m_new;
         l *= alpha;
-        // P = 2^(t - m_ref), written as packed bf16 over the first 64 columns of S.
+        if (warp_need && j > 0) {
+          // O holds P V up to tile j-1 (complete: S(j) was committed after that product);
+          // bring it to the new reference max before this tile's P is published.
+          if (!mbar_wait(pv_done + i, (pvcnt + j - 1) & 1)) { ok = false; break; }
+          tc_fence_after();
+#pragma unroll 1
+          for (int cc = 0; cc < D / 16; ++cc) {
+            uint32_t ov[16];
+            tmem_ld16(tO + 16 * cc, ov);
+            tmem_wait_ld();
+#pragma unroll
+            for (int e = 0; e < 16; ++e) ov[e] = __float_as_uint(__uint_as_float(ov[e]) * alpha);
+            tmem_st16(tO + 16 * cc, ov);
+          }
+          tmem_wait_st();
+        }
+        // P = 2^(t - m_ref) as packed bf16 over the first 64 columns of S, published in two
+        // halves of 64 keys so the P V product starts on the first while the second is made.
         const float ms = (m_ref == -INFINITY) ? 0.f : m_ref;
-        float ls0 = 0.f, ls1 = 0.f;
+        const uint64_t tau2 = f2(tau, tau), nms2 = f2(-ms, -ms);
+        uint64_t lsum[2] = {f2(0.f, 0.f), f2(0.f, 0.f)};
 #pragma unroll
         for (int half = 0; half < 2; ++half) {
           uint32_t pk[32];
 #pragma unroll
-          for (int c = 0; c < 32; ++c) {
-            const float p0 = ex2_approx(fmaf(s[64 * half + 2 * c], tau, -ms));
-            const float p1 = ex2_approx(fmaf(s[64 * half + 2 * c + 1], tau, -ms));
-            ls0 += p0;
-            ls1 += p1;
-            pk[c] = pack_bf16x2(p0, p1);
+          for (int e = 0; e < 32; ++e) {
+            const int g = 32 * half + e;  // column pair
+            float x0, x1, p0, p1;
+            f2_split(f2_fma(f2(s[2 * g], s[2 * g + 1]), tau2, nms2), x0, x1);
+            if (((kEmuPairMask >> (g & 7)) & 1u) && !need_mask) {
+              exp2_poly_x2(x0, x1, p0, p1);
+            } else {
+              p0 = ex2_approx(x0);
+              p1 = ex2_approx(x1);
+            }
+            lsum[g & 1] = f2_add(lsum[g & 1], f2(p0, p1));
+            pk[e] = ((kIntPackPairMask >> (g & 7)) & 1u) ? pack_bf16x2_int(p0, p1) : pack_bf16x2(p0, p1);
           }
           tmem_st32(tS + 32 * half, pk);
+          tmem_wait_st();
+          tc_fence_before();
+          mbar_arrive(p_half + 2 * i + half);
         }
-        l += ls0 + ls1;
-        if (warp_need && j > 0) {
-          // O holds P V up to tile j-1 (complete: S(j) was committed after that product);
-          // bring it to the new reference max.
-          if (!mbar_wait(pv_done + i, (pvcnt + j - 1) & 1)) { ok = false; break; }
-          tc_fence_after();
-#pragma unroll
-          for (int c = 0; c < D / 32; ++c) {
-            uint32_t ov[32];
-            tmem_ld32(tO + 32 * c, ov);
-            tmem_wait_ld();
-#pragma unroll
-            for (int e = 0; e < 32; ++e) ov[e] = __float_as_uint(__uint_as_float(ov[e]) * alpha);
-            tmem_st32(tO + 32 * c, ov);
-          }
-        }
-        tmem_wait_st();
-        tc_fence_before();
-        mbar_arrive(p_full + i);
+        float la, lb, lc, ld;
+        f2_split(lsum[0], la, lb);
+        f2_split(lsum[1], lc, ld);
+        l += (la + lb) + (lc + ld);
       }
       if (!ok) break;
 
