@@ -18,7 +18,8 @@ FA_OK, FA_ERR_INVALID_ARG, FA_ERR_UNSUPPORTED, FA_ERR_WORKSPACE, FA_ERR_CUDA, FA
 FA_BF16, FA_F32 = 0, 1
 
 EXPORTED = ("fa_fwd", "fa_fwd_workspace_size", "fa_decode", "fa_decode_workspace_size", "fa_decode_noalloc",
-            "fa_last_device_error", "fa_status_string", "fa_device_sm_count")
+            "fa_decode_paged", "fa_decode_paged_workspace_size", "fa_last_device_error", "fa_status_string",
+            "fa_device_sm_count")
 FA_DECODE_NOALLOC_SCRATCH_BYTES = 16 << 20
 
 
@@ -50,6 +51,10 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
     L.fa_decode_noalloc.restype = i
     L.fa_decode_workspace_size.argtypes = [i, i, i, i, i]
     L.fa_decode_workspace_size.restype = sz
+    L.fa_decode_paged.argtypes = [vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, i, i, f, i, vp, sz, vp]
+    L.fa_decode_paged.restype = i
+    L.fa_decode_paged_workspace_size.argtypes = [i, i, i, i, i, i, i]
+    L.fa_decode_paged_workspace_size.restype = sz
     L.fa_last_device_error.argtypes = [vp]
     L.fa_last_device_error.restype = i
     L.fa_status_string.argtypes = [i]
@@ -122,6 +127,20 @@ def fa_decode_workspace_size(B, Hq, Lmax, d, split_len) -> int:
     return int(load().fa_decode_workspace_size(int(B), int(Hq), int(Lmax), int(d), int(split_len)))
 
 
+def fa_decode_paged(q, k_pages, v_pages, block_table, seqlens, o, lse, B, Hq, Hkv, num_pages, page_size,
+                    max_pages_per_seq, d, scale, split_len, workspace, workspace_bytes, stream=None) -> None:
+    st = load().fa_decode_paged(_ptr(q), _ptr(k_pages), _ptr(v_pages), _ptr(block_table), _ptr(seqlens), _ptr(o),
+                                _ptr(lse), int(B), int(Hq), int(Hkv), int(num_pages), int(page_size),
+                                int(max_pages_per_seq), int(d), float(scale), int(split_len), _ptr(workspace),
+                                int(workspace_bytes), _stream(stream))
+    _check(st, "fa_decode_paged")
+
+
+def fa_decode_paged_workspace_size(B, Hq, Hkv, max_pages_per_seq, page_size, d, split_len) -> int:
+    return int(load().fa_decode_paged_workspace_size(int(B), int(Hq), int(Hkv), int(max_pages_per_seq),
+                                                     int(page_size), int(d), int(split_len)))
+
+
 def fa_last_device_error(stream=None) -> int:
     return int(load().fa_last_device_error(_stream(stream)))
 
@@ -179,4 +198,28 @@ def decode(q, kcache, vcache, seqlens=None, scale=None, split_len=1024, out=None
         workspace = torch.empty(max(ws_bytes, 1), dtype=torch.uint8, device=q.device)
     fa_decode(q, kcache, vcache, seqlens, out, lse, B, Hq, Hkv, Lmax, d, scale, split_len, workspace, ws_bytes,
               stream)
+    return out, lse
+
+
+def decode_paged(q, k_pages, v_pages, block_table, seqlens, scale=None, split_len=1024, out=None, lse=None,
+                 workspace=None, stream=None):
+    """O [B,Hq,d], lse [B,Hq] for one query token per sequence over a page pool
+    [num_pages, page_size, Hkv, d] addressed by block_table [B, max_pages] (int32) and
+    seqlens [B] (int32).  A workspace passed in must have been zero-filled once (its arrival
+    counters); calls leave it ready for the next call."""
+    import torch
+    B, Hq, d = q.shape
+    num_pages, page_size, Hkv = k_pages.shape[0], k_pages.shape[1], k_pages.shape[2]
+    maxp = block_table.shape[1]
+    if scale is None:
+        scale = d ** -0.5
+    if out is None:
+        out = torch.empty((B, Hq, d), dtype=torch.bfloat16, device=q.device)
+    if lse is None:
+        lse = torch.empty((B, Hq), dtype=torch.float32, device=q.device)
+    ws_bytes = fa_decode_paged_workspace_size(B, Hq, Hkv, maxp, page_size, d, split_len)
+    if workspace is None:
+        workspace = torch.zeros(max(ws_bytes, 1), dtype=torch.uint8, device=q.device)
+    fa_decode_paged(q, k_pages, v_pages, block_table, seqlens, out, lse, B, Hq, Hkv, num_pages, page_size, maxp, d,
+                    scale, split_len, workspace, ws_bytes, stream)
     return out, lse

@@ -105,7 +105,7 @@ fa_status launch_decode(const void* kc, const void* vc, const DecParams& prm, cu
   const int64_t rows = (int64_t)prm.B * prm.Lmax;
   if (!make_map(&mk, kc, D, prm.Hkv, rows, kDecKeys) || !make_map(&mv, vc, D, prm.Hkv, rows, kDecKeys))
     return FA_ERR_CUDA;
-  auto ks = fa_decode_split_kernel<D>;
+  auto ks = fa_decode_split_kernel<D, false>;
   const int smem = DecCfg<D>::kSmemBytes;
   if (set_smem(ks, smem) != cudaSuccess) return FA_ERR_CUDA;
   dim3 grid(prm.nsplit, prm.Hkv, prm.B);
@@ -113,6 +113,20 @@ fa_status launch_decode(const void* kc, const void* vc, const DecParams& prm, cu
   if (cudaGetLastError() != cudaSuccess) return FA_ERR_CUDA;
   const int nbh = prm.B * prm.Hq;
   fa_decode_combine_kernel<D><<<(nbh + 3) / 4, 128, 0, st>>>(prm);
+  return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+}
+
+template <int D>
+fa_status launch_decode_paged(const void* kp, const void* vp, const DecParams& prm, cudaStream_t st) {
+  CUtensorMap mk, mv;
+  const int64_t rows = (int64_t)prm.num_pages << prm.page_shift;
+  if (!make_map(&mk, kp, D, prm.Hkv, rows, prm.page_box) || !make_map(&mv, vp, D, prm.Hkv, rows, prm.page_box))
+    return FA_ERR_CUDA;
+  auto ks = fa_decode_split_kernel<D, true>;
+  const int smem = DecCfg<D>::kSmemBytes;
+  if (set_smem(ks, smem) != cudaSuccess) return FA_ERR_CUDA;
+  dim3 grid(prm.nsplit, prm.Hkv, prm.B);
+  ks<<<grid, kDecThreads, smem, st>>>(mk, mv, prm);
   return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
 
@@ -259,6 +273,69 @@ fa_status fa_decode(const void* q, const void* kcache, const void* vcache, const
   return d == 64 ? launch_decode<64>(kcache, vcache, prm, st) : launch_decode<128>(kcache, vcache, prm, st);
 }
 
+size_t fa_decode_paged_workspace_size(int B, int Hq, int Hkv, int max_pages_per_seq, int page_size, int d,
+                                      int split_len) {
+  if (B <= 0 || Hq <= 0 || Hkv <= 0 || max_pages_per_seq <= 0 || page_size <= 0 || d <= 0 || split_len <= 0)
+    return 0;
+  const int64_t lmax = (int64_t)max_pages_per_seq * page_size;
+  if (lmax >= (int64_t(1) << 31)) return 0;
+  return align_up((size_t)B * Hkv * 4, 256) + fa_decode_workspace_size(B, Hq, (int)lmax, d, split_len);
+}
+
+fa_status fa_decode_paged(const void* q, const void* k_pages, const void* v_pages, const int32_t* block_table,
+                          const int32_t* seqlens, void* o, float* lse, int B, int Hq, int Hkv, int num_pages,
+                          int page_size, int max_pages_per_seq, int d, float scale, int split_len, void* workspace,
+                          size_t workspace_bytes, void* stream) {
+  if (!q || !k_pages || !v_pages || !block_table || !seqlens || !o) return FA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k_pages) || !aligned16(v_pages) || !aligned16(o)) return FA_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(block_table) & 3u) != 0 || (reinterpret_cast<uintptr_t>(seqlens) & 3u) != 0)
+    return FA_ERR_INVALID_ARG;
+  if (B < 0 || Hq <= 0 || Hkv <= 0 || num_pages <= 0 || page_size <= 0 || max_pages_per_seq <= 0 || split_len <= 0)
+    return FA_ERR_INVALID_ARG;
+  if (!(scale > 0.f) || !std::isfinite(scale)) return FA_ERR_INVALID_ARG;
+  if ((page_size & (page_size - 1)) != 0) return FA_ERR_UNSUPPORTED;
+  if (page_size < 16) return FA_ERR_UNSUPPORTED;
+  if (Hq % Hkv != 0) return FA_ERR_UNSUPPORTED;
+  if (Hq / Hkv > 16) return FA_ERR_UNSUPPORTED;
+  if (d != 64 && d != 128) return FA_ERR_UNSUPPORTED;
+  if (split_len % kDecKeys != 0) return FA_ERR_UNSUPPORTED;
+  if ((int64_t)num_pages * page_size >= (int64_t(1) << 31)) return FA_ERR_UNSUPPORTED;
+  const int64_t lmax = (int64_t)max_pages_per_seq * page_size;
+  if (lmax >= (int64_t(1) << 31)) return FA_ERR_UNSUPPORTED;
+  if (B == 0) return FA_OK;
+  const int nsplit = (int)((lmax + split_len - 1) / split_len);
+  if (nsplit > 65535 || Hkv > 65535 || B > 65535) return FA_ERR_UNSUPPORTED;
+  const size_t need = fa_decode_paged_workspace_size(B, Hq, Hkv, max_pages_per_seq, page_size, d, split_len);
+  if (!workspace || workspace_bytes < need || !aligned16(workspace)) return FA_ERR_WORKSPACE;
+  const size_t parts = (size_t)B * Hq * nsplit;
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  DecParams prm{};
+  prm.q = static_cast<const __nv_bfloat16*>(q);
+  prm.seqlens = seqlens;
+  prm.o = static_cast<__nv_bfloat16*>(o);
+  prm.lse = lse;
+  prm.counters = reinterpret_cast<uint32_t*>(ws);
+  ws += align_up((size_t)B * Hkv * 4, 256);
+  prm.ws_acc = reinterpret_cast<float*>(ws);
+  prm.ws_ml = reinterpret_cast<float*>(ws + align_up(parts * d * 4, 256));
+  prm.block_table = block_table;
+  prm.max_pages = max_pages_per_seq;
+  prm.page_shift = __builtin_ctz((unsigned)page_size);
+  prm.page_box = std::min(page_size, kDecKeys);
+  prm.num_pages = num_pages;
+  prm.B = B;
+  prm.Hq = Hq;
+  prm.Hkv = Hkv;
+  prm.G = Hq / Hkv;
+  prm.Lmax = (int)lmax;
+  prm.split_len = split_len;
+  prm.nsplit = nsplit;
+  prm.tau = (float)((double)scale * 1.4426950408889634074);
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  return d == 64 ? launch_decode_paged<64>(k_pages, v_pages, prm, st)
+                 : launch_decode_paged<128>(k_pages, v_pages, prm, st);
+}
+
 fa_status fa_last_device_error(void* stream) {
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   if (cudaStreamSynchronize(st) != cudaSuccess) return FA_ERR_CUDA;
@@ -267,7 +344,7 @@ fa_status fa_last_device_error(void* stream) {
   if (w != 0) {
     const unsigned int zero = 0;
     if (cudaMemcpyToSymbol(g_error_word, &zero, sizeof(zero)) != cudaSuccess) return FA_ERR_CUDA;
-    return FA_ERR_TIMEOUT;
+    return (w & kErrTimeout) ? FA_ERR_TIMEOUT : FA_ERR_INVALID_ARG;
   }
   return FA_OK;
 }

@@ -9,6 +9,15 @@
 // rule of "FlashAttention notes" section 4 (m = max m_s, l = sum 2^(m_s - m) l_s, and the
 // accumulators with the same weights) ("FlashAttention-3 (FA-3)", section 4, FlashDecoding).
 //
+// Paged caches ("LLM basics: from Attention to FlashAttention", chapter 2 section 8,
+// PagedAttention): the cache is a pool of fixed-size pages, and a per-sequence block table
+// maps logical page t / page_size of a sequence to a physical page, so token t sits at row
+// t % page_size of that page.  The paged kernel fetches each 64-row stage as whole pages
+// (or one 64-row part of a larger page) through the table, and merges the splits itself:
+// every split CTA publishes its partial, counts itself in on a per-(sequence, KV head)
+// counter, and the CTA that arrives last merges all partials of that group (no CTA waits
+// for another, and no second launch).  A sequence that fits one split skips the partial.
+//
 // The split kernel is bound by HBM bandwidth: K and V are read once.  Tiles of 64 cache rows
 // arrive by TMA (128-byte swizzle, evict-first) in a 3- or 4-stage ring fed by a producer
 // warp; four compute warps each take 16 of the 64 rows.  The G <= 16 query heads of the
@@ -27,9 +36,15 @@ struct DecParams {
   float* lse;
   float* ws_acc;  // [B, Hq, nsplit, D]
   float* ws_ml;   // [B, Hq, nsplit, 2]  (m in base-2 units, l)
+  // paged caches only
+  const int32_t* block_table;  // [B, max_pages]
+  uint32_t* counters;          // [B, Hkv] split arrivals; zero between calls
+  int max_pages, page_shift, page_box, num_pages;
   int B, Hq, Hkv, G, Lmax, split_len, nsplit;
   float tau;
 };
+
+constexpr unsigned int kErrBadPage = 2u;  // a block-table entry outside [0, num_pages)
 
 constexpr int kDecKeys = 64;  // cache rows per stage
 constexpr int kDecComputeWarps = 4;
@@ -42,6 +57,8 @@ struct DecCfg {
   static constexpr int kStageBytes = 2 * kHalfBytes;
   static constexpr int kStages = (D == 128) ? 3 : 4;
   static constexpr int kSmemBytes = 1024 + kStages * kStageBytes + 2 * kStages * 8 + 64;
+  static_assert(kStages * kStageBytes >= (kDecComputeWarps * 16 * D + 2 * kDecComputeWarps * 16 + 32) * 4,
+                "the merge scratch must fit in the ring");
 };
 
 __device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3) {
@@ -75,7 +92,22 @@ __device__ __forceinline__ int dec_seqlen(const DecParams& p, int b) {
   return max(0, min(L, p.Lmax));
 }
 
-template <int D>
+// Writes o (bf16) and lse of query head h of sequence b from the merged numerator a / l and
+// the base-2 max m.  An empty row (l = 0) gives o = 0 and lse = -inf.
+__device__ __forceinline__ void dec_store_row4(const DecParams& p, int b, int h, int col, float4 a, float m, float l,
+                                               int D) {
+  const float inv = l > 0.f ? 1.f / l : 0.f;
+  uint2 w;
+  w.x = pack_bf16x2(a.x * inv, a.y * inv);
+  w.y = pack_bf16x2(a.z * inv, a.w * inv);
+  *reinterpret_cast<uint2*>(p.o + ((size_t)b * p.Hq + h) * D + col) = w;
+  if (col == 0 && p.lse != nullptr) p.lse[(size_t)b * p.Hq + h] = l > 0.f ? (m + log2f(l)) * kLn2 : -INFINITY;
+}
+
+// PAGED = false: contiguous caches [B, Lmax, Hkv, D]; partials of every split go to the
+// workspace and fa_decode_combine_kernel merges them.  PAGED = true: page pool
+// [num_pages, page_size, Hkv, D] through the block table, merged in this kernel.
+template <int D, bool PAGED>
 __global__ void __launch_bounds__(kDecThreads)
     fa_decode_split_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                            const DecParams p) {
@@ -84,7 +116,17 @@ __global__ void __launch_bounds__(kDecThreads)
   const int split = blockIdx.x, kvh = blockIdx.y, b = blockIdx.z;
   const int seqlen = dec_seqlen(p, b);
   const int key_begin = split * p.split_len;
-  if (key_begin >= seqlen) return;  // empty split: the combine kernel never reads it
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int G = p.G;
+  const int h0 = kvh * G;
+  if (key_begin >= seqlen) {
+    // Empty split.  Unpaged, the combine kernel never reads it.  Paged, an empty sequence
+    // still needs its output, which the first split writes.
+    if (PAGED && split == 0 && warp < kDecComputeWarps)
+      for (int idx = threadIdx.x; idx < G * (D / 4); idx += kDecComputeWarps * 32)
+        dec_store_row4(p, b, h0 + idx / (D / 4), 4 * (idx % (D / 4)), make_float4(0.f, 0.f, 0.f, 0.f), 0.f, 0.f, D);
+    return;
+  }
   const int nkeys = min(p.split_len, seqlen - key_begin);
   const int nst = (nkeys + kDecKeys - 1) / kDecKeys;
 
@@ -92,8 +134,7 @@ __global__ void __launch_bounds__(kDecThreads)
   uint8_t* ring = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* full = reinterpret_cast<uint64_t*>(ring + NS * C::kStageBytes);
   uint64_t* empty = full + NS;
-
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  uint32_t* last_flag = reinterpret_cast<uint32_t*>(empty + NS);
   if (threadIdx.x == 0) {
     for (int s = 0; s < NS; ++s) {
       mbar_init(full + s, 1);
@@ -115,10 +156,33 @@ __global__ void __launch_bounds__(kDecThreads)
         if (s >= NS && !mbar_wait(empty + slot, ((s / NS) - 1) & 1)) break;
         mbar_arrive_expect_tx(full + slot, C::kStageBytes);
         uint8_t* st = ring + slot * C::kStageBytes;
-        for (int c = 0; c < D / 64; ++c) {
-          tma_load_3d_hint(st + c * C::kPanelBytes, &tmK, c * 64, kvh, row_base + s * kDecKeys, full + slot, pol);
-          tma_load_3d_hint(st + C::kHalfBytes + c * C::kPanelBytes, &tmV, c * 64, kvh, row_base + s * kDecKeys,
-                           full + slot, pol);
+        if (!PAGED) {
+          for (int c = 0; c < D / 64; ++c) {
+            tma_load_3d_hint(st + c * C::kPanelBytes, &tmK, c * 64, kvh, row_base + s * kDecKeys, full + slot, pol);
+            tma_load_3d_hint(st + C::kHalfBytes + c * C::kPanelBytes, &tmV, c * 64, kvh, row_base + s * kDecKeys,
+                             full + slot, pol);
+          }
+        } else {
+          // page_box = min(page_size, 64) rows per copy; a stage never straddles a page
+          // boundary inside one copy.  Copies past the sequence end re-read its last page
+          // (those rows are masked and their V rows zeroed before use).
+          const int box = p.page_box;
+          const int ps = 1 << p.page_shift;
+          for (int t = 0; t < kDecKeys; t += box) {
+            int tok = key_begin + s * kDecKeys + t;
+            if (tok >= seqlen) tok = (seqlen - 1) & ~(box - 1);
+            int page = __ldg(p.block_table + (size_t)b * p.max_pages + (tok >> p.page_shift));
+            if (page < 0 || page >= p.num_pages) {
+              atomicOr(&g_error_word, kErrBadPage);
+              page = 0;
+            }
+            const int row = page * ps + (tok & (ps - 1));
+            for (int c = 0; c < D / 64; ++c) {
+              tma_load_3d_hint(st + c * C::kPanelBytes + t * 128, &tmK, c * 64, kvh, row, full + slot, pol);
+              tma_load_3d_hint(st + C::kHalfBytes + c * C::kPanelBytes + t * 128, &tmV, c * 64, kvh, row,
+                               full + slot, pol);
+            }
+          }
         }
       }
     }
@@ -127,8 +191,6 @@ __global__ void __launch_bounds__(kDecThreads)
 
   // -------------------------------------------------------------- compute warps
   const int g = lane >> 2, tig = lane & 3;
-  const int G = p.G;
-  const int h0 = kvh * G;
   // A fragments of q (rows = the group's query heads, zero beyond G)
   uint32_t qa[D / 16][4];
   {
@@ -169,7 +231,9 @@ __global__ void __launch_bounds__(kDecThreads)
       mma_bf16_16816(sc[0], qa[kk], b0, b1);
       mma_bf16_16816(sc[1], qa[kk], b2, b3);
     }
-    // mask rows of the cache at or beyond the sequence length
+    // Mask rows of the cache at or beyond the sequence length, and zero their V rows: those
+    // rows are unused cache slots whose contents are arbitrary (0 * NaN would poison O).
+    // Each warp reads only its own 16 V rows, so a warp-local barrier orders the zeroing.
     const int kglob0 = key_begin + s * kDecKeys + key_lo;
     if (kglob0 + 16 > seqlen) {
 #pragma unroll
@@ -177,6 +241,15 @@ __global__ void __launch_bounds__(kDecThreads)
 #pragma unroll
         for (int e = 0; e < 4; ++e)
           if (kglob0 + nt * 8 + 2 * tig + (e & 1) >= seqlen) sc[nt][e] = -INFINITY;
+      uint8_t* vrows = ring + slot * C::kStageBytes + C::kHalfBytes;
+#pragma unroll
+      for (int u = lane; u < 16 * (D / 64) * 8; u += 32) {
+        const int r = u & 15, c = u >> 4;  // row within the warp's 16, 16-byte unit of the row
+        if (kglob0 + r >= seqlen)
+          *reinterpret_cast<uint4*>(vrows + (c >> 3) * C::kPanelBytes + (key_lo + r) * 128 + (c & 7) * 16) =
+              make_uint4(0u, 0u, 0u, 0u);
+      }
+      __syncwarp();
     }
     // online softmax update for rows g (e = 0, 1) and g + 8 (e = 2, 3)
     float alpha[2], ms[2];
@@ -217,6 +290,11 @@ __global__ void __launch_bounds__(kDecThreads)
       mma_bf16_16816(acc[2 * qd], pa, b0, b1);
       mma_bf16_16816(acc[2 * qd + 1], pa, b2, b3);
     }
+    // The slot is refilled by TMA (the async proxy) once every warp has arrived.  The warp's
+    // ldmatrix reads of it are generic-proxy accesses, so a cross-proxy fence orders them
+    // before that refill; without it a refill was seen to overwrite V while a warp still
+    // read it (two CTAs per SM, about one run in a few hundred).
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
     __syncwarp();
     if (lane == 0) mbar_arrive(empty + slot);
   }
@@ -253,25 +331,93 @@ __global__ void __launch_bounds__(kDecThreads)
   }
   asm volatile("bar.sync 1, %0;" ::"n"(kDecComputeWarps * 32) : "memory");
   const size_t part0 = ((size_t)b * p.Hq + h0) * p.nsplit + split;  // partial of head h0
-  for (int idx = threadIdx.x; idx < G * D; idx += kDecComputeWarps * 32) {
-    const int row = idx / D, col = idx - row * D;
+  const int ns_b = (seqlen + p.split_len - 1) / p.split_len;       // splits of this sequence
+  for (int idx = threadIdx.x; idx < G * (D / 4); idx += kDecComputeWarps * 32) {
+    const int row = idx / (D / 4), col = 4 * (idx - row * (D / 4));
     float M = -INFINITY;
 #pragma unroll
     for (int w = 0; w < kDecComputeWarps; ++w) M = fmaxf(M, sm_m[w * 16 + row]);
-    float L = 0.f, A = 0.f;
+    float L = 0.f;
+    float4 A = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
     for (int w = 0; w < kDecComputeWarps; ++w) {
       const float mw = sm_m[w * 16 + row];
       const float e = (mw == -INFINITY) ? 0.f : ex2_approx(mw - M);
       L += e * sm_l[w * 16 + row];
-      A += e * sm_o[(w * 16 + row) * D + col];
+      const float4 x = *reinterpret_cast<const float4*>(sm_o + (w * 16 + row) * D + col);
+      A.x += e * x.x;
+      A.y += e * x.y;
+      A.z += e * x.z;
+      A.w += e * x.w;
+    }
+    if (PAGED && ns_b == 1) {  // the only split of its sequence: the result is final
+      dec_store_row4(p, b, h0 + row, col, A, M, L, D);
+      continue;
     }
     const size_t part = part0 + (size_t)row * p.nsplit;
-    p.ws_acc[part * D + col] = A;
+    *reinterpret_cast<float4*>(p.ws_acc + part * D + col) = A;
     if (col == 0) {
       p.ws_ml[part * 2] = M;
       p.ws_ml[part * 2 + 1] = L;
     }
+  }
+  if (!PAGED || ns_b == 1) return;
+
+  // Count this split in; the last of the sequence's splits to arrive merges them all.  Each
+  // writer fences its partial before the CTA barrier, and the counting thread's atomic is
+  // ordered after that barrier, so a CTA that sees the final count sees every partial.
+  __threadfence();
+  asm volatile("bar.sync 1, %0;" ::"n"(kDecComputeWarps * 32) : "memory");
+  uint32_t* counter = p.counters + (size_t)b * p.Hkv + kvh;
+  if (threadIdx.x == 0) {
+    const uint32_t before = atomicAdd(counter, 1u);
+    const bool last = before + 1 == (uint32_t)ns_b;
+    if (last) *counter = 0u;  // every split of this call has counted; ready for the next call
+    __threadfence();
+    *last_flag = last ? 1u : 0u;
+  }
+  asm volatile("bar.sync 1, %0;" ::"n"(kDecComputeWarps * 32) : "memory");
+  if (*last_flag == 0u) return;
+
+  // Merge ("FlashAttention notes", section 4): m = max_s m_s, l = sum_s 2^(m_s - m) l_s,
+  // o = sum_s 2^(m_s - m) acc_s / l.  Partials were written by other SMs: read through L2.
+  float* sm_M = sm_l + kDecComputeWarps * 16;  // [16]
+  float* sm_L = sm_M + 16;                     // [16]
+  const size_t bh0 = ((size_t)b * p.Hq + h0) * p.nsplit;
+  for (int row = warp; row < G; row += kDecComputeWarps) {
+    const float* ml = p.ws_ml + (bh0 + (size_t)row * p.nsplit) * 2;
+    float M = -INFINITY;
+    for (int s = lane; s < ns_b; s += 32) M = fmaxf(M, __ldcg(ml + 2 * s));
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
+    float L = 0.f;
+    for (int s = lane; s < ns_b; s += 32) {
+      const float ms = __ldcg(ml + 2 * s);
+      L += (ms == -INFINITY) ? 0.f : ex2_approx(ms - M) * __ldcg(ml + 2 * s + 1);
+    }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) L += __shfl_xor_sync(0xffffffffu, L, off);
+    if (lane == 0) {
+      sm_M[row] = M;
+      sm_L[row] = L;
+    }
+  }
+  asm volatile("bar.sync 1, %0;" ::"n"(kDecComputeWarps * 32) : "memory");
+  for (int idx = threadIdx.x; idx < G * (D / 4); idx += kDecComputeWarps * 32) {
+    const int row = idx / (D / 4), col = 4 * (idx - row * (D / 4));
+    const size_t base = bh0 + (size_t)row * p.nsplit;
+    const float M = sm_M[row];
+    float4 A = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int s = 0; s < ns_b; ++s) {
+      const float ms = __ldcg(p.ws_ml + (base + s) * 2);
+      const float e = (ms == -INFINITY) ? 0.f : ex2_approx(ms - M);
+      const float4 x = __ldcg(reinterpret_cast<const float4*>(p.ws_acc + (base + s) * D + col));
+      A.x += e * x.x;
+      A.y += e * x.y;
+      A.z += e * x.z;
+      A.w += e * x.w;
+    }
+    dec_store_row4(p, b, h0 + row, col, A, M, sm_L[row], D);
   }
 }
 

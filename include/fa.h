@@ -13,6 +13,7 @@
  *   fa_decode  single-token decode over a KV cache, split along the cache; the partial
  *              results are merged with the same m/l rule ("FlashAttention-3 (FA-3)",
  *              section 4 "FlashDecoding"; "FlashAttention notes", section 4).
+ *   fa_decode_paged  the same decode over a paged cache addressed through a block table.
  *
  * Conventions for every entry point:
  *   - All tensor pointers are DEVICE pointers owned by the caller.  The library never
@@ -126,9 +127,44 @@ FA_EXPORT fa_status fa_decode_noalloc(const void* q, const void* kcache, const v
                                       void* o, float* lse, int B, int Hq, int Hkv, int Lmax, int d, float scale,
                                       int split_len, void* stream);
 
+/* Split-KV decode over a paged KV cache ("LLM basics: from Attention to FlashAttention",
+ * chapter 2 section 8, PagedAttention: fixed-size pages of the cache, mapped from each
+ * sequence's logical pages by a block table), with the split merge done inside the same
+ * launch by the last split of each (sequence, KV head) to finish.
+ *
+ * q [B, Hq, d] bf16; k_pages and v_pages [num_pages, page_size, Hkv, d] bf16 (the page
+ * pool); block_table: device int32 [B, max_pages_per_seq], entry (b, t) = the physical page
+ * holding tokens t*page_size .. (t+1)*page_size - 1 of sequence b; seqlens: device int32 [B],
+ * required, 0 <= seqlens[b] <= max_pages_per_seq * page_size (larger values are clamped).
+ * Only the first ceil(seqlens[b] / page_size) entries of row b are read; pages may be
+ * shared between sequences and appear in any order.  o [B, Hq, d] bf16; lse [B, Hq] fp32
+ * (may be NULL).  Token j of sequence b takes part iff j < seqlens[b]; an empty sequence gets
+ * o = 0 and lse = -inf.  Rows of a page beyond a sequence's length may hold anything
+ * (NaN included): they are masked and never multiply into o.
+ * page_size: a power of two >= 16.  split_len: a multiple of 64.  Hq / Hkv <= 16; d 64 or
+ * 128; q, the pages and o 16-byte aligned; block_table and seqlens 4-byte aligned;
+ * num_pages * page_size < 2^31.
+ * A block-table entry outside [0, num_pages) is read as page 0 and recorded on the device;
+ * fa_last_device_error then returns FA_ERR_INVALID_ARG.
+ * workspace: at least fa_decode_paged_workspace_size(...) bytes.  Its first
+ * 4 * B * Hkv bytes (rounded up to 256) are arrival counters that MUST be zero before the
+ * first call with this workspace (e.g. allocate it zero-filled); every call that completes
+ * leaves them zero again, so the same workspace serves later calls without clearing.  After
+ * a call that reported FA_ERR_TIMEOUT, zero it again.  Calls sharing a workspace must not
+ * overlap on the GPU. */
+FA_EXPORT fa_status fa_decode_paged(const void* q, const void* k_pages, const void* v_pages,
+                                    const int32_t* block_table, const int32_t* seqlens, void* o, float* lse, int B,
+                                    int Hq, int Hkv, int num_pages, int page_size, int max_pages_per_seq, int d,
+                                    float scale, int split_len, void* workspace, size_t workspace_bytes,
+                                    void* stream);
+
+FA_EXPORT size_t fa_decode_paged_workspace_size(int B, int Hq, int Hkv, int max_pages_per_seq, int page_size, int d,
+                                                int split_len);
+
 /* Waits for `stream`, then returns FA_ERR_TIMEOUT if any kernel of this library recorded a
- * device-side timeout since the previous call (and clears the record), FA_ERR_CUDA if the
- * stream reports an error, else FA_OK. */
+ * device-side timeout since the previous call, else FA_ERR_INVALID_ARG if a kernel recorded
+ * an invalid device-side input (a block-table entry out of range), and clears the record;
+ * FA_ERR_CUDA if the stream reports an error; else FA_OK. */
 FA_EXPORT fa_status fa_last_device_error(void* stream);
 
 /* Static description of a status code. */

@@ -151,6 +151,30 @@ class Oracle:
                                 kv_lens=seqlens, nthreads=nthreads)
         return o.reshape(B, Hq, d), lse.reshape(B, Hq)
 
+    @staticmethod
+    def gather_pages(pages, block_table, seqlens, page_size):
+        """Contiguous per-sequence cache [B, Lmax, H, d] from a page pool [P, page_size, H, d]
+        ("LLM basics: from Attention to FlashAttention", chapter 2 section 8, PagedAttention:
+        a sequence's logical page t is the physical page block_table[b, t]; token j of the
+        sequence is row j % page_size of its logical page j // page_size).  Rows at or past
+        seqlens[b] are left zero (decode never reads them)."""
+        pages = np.asarray(pages)
+        table = np.asarray(block_table)
+        B, maxp = table.shape
+        H, d = pages.shape[2], pages.shape[3]
+        out = np.zeros((B, maxp * page_size, H, d), dtype=pages.dtype)
+        for b in range(B):
+            for j in range(int(seqlens[b])):
+                out[b, j] = pages[table[b, j // page_size], j % page_size]
+        return out
+
+    def decode_paged(self, q, k_pages, v_pages, block_table, seqlens, page_size, scale, nthreads=0):
+        """Decode over a paged cache: each sequence's cache is read through its block table
+        (gather_pages), then the plain decode definition applies."""
+        kc = self.gather_pages(k_pages, block_table, seqlens, page_size)
+        vc = self.gather_pages(v_pages, block_table, seqlens, page_size)
+        return self.decode(q, kc, vc, np.asarray(seqlens), scale, nthreads=nthreads)
+
     def hardware_threads(self) -> int:
         return int(self.lib.oracle_hardware_threads())
 

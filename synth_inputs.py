@@ -33,7 +33,7 @@ _M1 = np.uint64(0xBF58476D1CE4E5B9)
 _M2 = np.uint64(0x94D049BB133111EB)
 
 # tensor ids of the streams
-Q, K, V, KCACHE, VCACHE, LENGTHS = 1, 2, 3, 4, 5, 6
+Q, K, V, KCACHE, VCACHE, LENGTHS, PAGES = 1, 2, 3, 4, 5, 6, 7
 
 
 def _mix(z: np.ndarray) -> np.ndarray:
@@ -123,6 +123,32 @@ def cu_seqlens(lengths) -> np.ndarray:
     return cu
 
 
+def permutation(seed: int, tensor_id: int, n: int) -> np.ndarray:
+    """A permutation of 0..n-1: the indices that sort n words of the stream (stable)."""
+    return np.argsort(words(stream_key(seed, tensor_id), 0, n), kind="stable").astype(np.int64)
+
+
+def page_layout(seed: int, lengths, page_size: int, extra_pages: int = 0, max_pages: int | None = None):
+    """Physical page placement for a paged KV cache.
+
+    Sequence b needs ceil(lengths[b] / page_size) pages.  All needed pages plus
+    `extra_pages` spare ones form the pool; the pool is shuffled by `permutation` (stream
+    PAGES) and handed out in order, sequence by sequence.  Returns (block_table int32
+    [B, max_pages] with -1 in entries a sequence does not use, num_pages)."""
+    lengths = np.asarray(lengths, dtype=np.int64)
+    need = (lengths + page_size - 1) // page_size
+    if max_pages is None:
+        max_pages = max(1, int(need.max()) if len(need) else 1)
+    num_pages = int(need.sum()) + extra_pages
+    perm = permutation(seed, PAGES, max(num_pages, 1))
+    table = np.full((len(lengths), max_pages), -1, dtype=np.int32)
+    nxt = 0
+    for b, n in enumerate(need):
+        table[b, :n] = perm[nxt:nxt + n]
+        nxt += int(n)
+    return table, max(num_pages, 1)
+
+
 # The benchmark workloads: every tensor is i.i.d. N(0,1); config k uses seed 1000 + k.
 WORKLOADS = {
     "single_head_f32": dict(B=1, Hq=1, Hkv=1, N=128, d=64, causal=0, dtype="f32", seed=1001),
@@ -131,4 +157,7 @@ WORKLOADS = {
     "varlen_gqa_causal": dict(nseq=16, len_lo=256, len_hi=8192, Hq=32, Hkv=8, d=128, causal=1,
                               dtype="bf16", seed=1004),
     "decode_split_kv": dict(B=8, Hq=64, Hkv=8, L=32768, d=128, split=1024, dtype="bf16", seed=1005),
+    # paged, ragged decode: 16 sequences of U{1..32768} tokens in 16-token pages, shuffled pool
+    "decode_paged_ragged": dict(B=16, Hq=64, Hkv=8, len_lo=1, len_hi=32768, page_size=16, d=128, split=1024,
+                                dtype="bf16", seed=1006),
 }

@@ -97,6 +97,40 @@ def test_decode_rejects_before_launch(lib):
     assert _dec_status(lib, sl=258) == fa.FA_ERR_INVALID_ARG
 
 
+def _paged_status(lib, **kw):
+    args = dict(q=256, kp=256, vp=256, bt=512, sl=768, o=256, lse=None, B=2, Hq=8, Hkv=2, P=10, ps=16, maxp=4,
+                d=128, scale=0.1, split=64, ws=256, wsb=1 << 30, st=None)
+    args.update(kw)
+    return lib.fa_decode_paged(args["q"], args["kp"], args["vp"], args["bt"], args["sl"], args["o"], args["lse"],
+                               args["B"], args["Hq"], args["Hkv"], args["P"], args["ps"], args["maxp"], args["d"],
+                               ctypes.c_float(args["scale"]), args["split"], args["ws"], args["wsb"], args["st"])
+
+
+def test_decode_paged_rejects_before_launch(lib):
+    assert _paged_status(lib, bt=None) == fa.FA_ERR_INVALID_ARG      # block table required
+    assert _paged_status(lib, sl=None) == fa.FA_ERR_INVALID_ARG      # lengths required
+    assert _paged_status(lib, bt=514) == fa.FA_ERR_INVALID_ARG       # misaligned table
+    assert _paged_status(lib, kp=264) == fa.FA_ERR_INVALID_ARG
+    assert _paged_status(lib, ps=24) == fa.FA_ERR_UNSUPPORTED        # not a power of two
+    assert _paged_status(lib, ps=8) == fa.FA_ERR_UNSUPPORTED         # below 16
+    assert _paged_status(lib, ps=0) == fa.FA_ERR_INVALID_ARG
+    assert _paged_status(lib, P=0) == fa.FA_ERR_INVALID_ARG
+    assert _paged_status(lib, maxp=0) == fa.FA_ERR_INVALID_ARG
+    assert _paged_status(lib, split=96) == fa.FA_ERR_UNSUPPORTED
+    assert _paged_status(lib, Hq=34, Hkv=2) == fa.FA_ERR_UNSUPPORTED
+    assert _paged_status(lib, P=1 << 27, ps=16) == fa.FA_ERR_UNSUPPORTED    # pool rows >= 2^31
+    assert _paged_status(lib, ws=None) == fa.FA_ERR_WORKSPACE
+    assert _paged_status(lib, wsb=64) == fa.FA_ERR_WORKSPACE
+    assert _paged_status(lib, B=0) == fa.FA_OK
+
+
+def test_decode_paged_workspace_holds_counters_and_partials(lib):
+    B, Hq, Hkv, maxp, ps, d, split = 16, 64, 8, 2048, 16, 128, 1024
+    n = fa.fa_decode_paged_workspace_size(B, Hq, Hkv, maxp, ps, d, split)
+    assert n >= B * Hkv * 4 + fa.fa_decode_workspace_size(B, Hq, maxp * ps, d, split)
+    assert fa.fa_decode_paged_workspace_size(0, Hq, Hkv, maxp, ps, d, split) == 0
+
+
 def test_empty_problems_are_noops(lib):
     # B == 0 or Nq == 0: valid, nothing launched
     assert _fwd_status(lib, B=0) == fa.FA_OK
