@@ -44,6 +44,7 @@ FALLBACK_BF16_TFLOPS = 1590.0
 
 FWD = si.WORKLOADS["gqa_causal_8k"]
 DEC = si.WORKLOADS["decode_split_kv"]
+PAGED = si.WORKLOADS["decode_paged_ragged"]
 
 
 def fwd_flops(w=FWD) -> float:
@@ -58,6 +59,14 @@ def fwd_bytes(w=FWD) -> float:
 
 def dec_kv_bytes(w=DEC) -> float:
     return 2.0 * w["B"] * w["L"] * w["Hkv"] * w["d"] * 2
+
+
+def paged_lengths(seed: int, w=PAGED) -> np.ndarray:
+    return si.uniform_ints(seed, si.LENGTHS, w["B"], w["len_lo"], w["len_hi"])
+
+
+def paged_kv_bytes(lengths, w=PAGED) -> float:
+    return 2.0 * float(np.sum(lengths)) * w["Hkv"] * w["d"] * 2
 
 
 def dec_flops(w=DEC) -> float:
@@ -230,6 +239,7 @@ def run_device(args):
 
     do_fwd = args.only in ("all", "fwd")
     do_dec = args.only in ("all", "dec")
+    do_paged = args.only in ("all", "paged")
     if not do_fwd:
         del q, k, v, o, lse
     wd = DEC
@@ -248,6 +258,27 @@ def run_device(args):
     ws = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
     h_do = torch.empty(do.shape, dtype=torch.bfloat16).pin_memory()
     dscale = 1.0 / math.sqrt(dd)
+
+    # ---- paged ragged decode: shuffled pool of 16-token pages, block table, lengths
+    wp = PAGED
+    pseed = replica_seed(wp["seed"], rank)
+    p_len = paged_lengths(pseed) if do_paged else np.ones(1, np.int64)
+    pB = len(p_len)
+    pps, pHq, pHkv, pd, psplit = wp["page_size"], wp["Hq"], wp["Hkv"], wp["d"], wp["split"]
+    table_np, npages = si.page_layout(pseed, p_len, pps)
+    p_q = torch.from_numpy(inputs("paged", pseed, si.Q, (pB, pHq, pd))).to(torch.bfloat16).to(dev)
+    p_k = torch.from_numpy(inputs("paged", pseed, si.KCACHE, (npages, pps, pHkv, pd))).to(torch.bfloat16).to(dev)
+    p_v = torch.from_numpy(inputs("paged", pseed, si.VCACHE, (npages, pps, pHkv, pd))).to(torch.bfloat16).to(dev)
+    p_table = torch.from_numpy(table_np).to(dev)
+    p_lens = torch.from_numpy(p_len.astype(np.int32)).to(dev)
+    p_o = torch.empty((pB, pHq, pd), dtype=torch.bfloat16, device=dev)
+    p_lse = torch.empty((pB, pHq), dtype=torch.float32, device=dev)
+    p_ws_bytes = fa.fa_decode_paged_workspace_size(pB, pHq, pHkv, table_np.shape[1], pps, pd, psplit)
+    p_ws = torch.zeros(p_ws_bytes, dtype=torch.uint8, device=dev)  # arrival counters start at zero
+
+    def call_paged():
+        fa.fa_decode_paged(p_q, p_k, p_v, p_table, p_lens, p_o, p_lse, pB, pHq, pHkv, npages, pps,
+                           table_np.shape[1], pd, 1.0 / math.sqrt(pd), psplit, p_ws, p_ws_bytes, st)
 
     def call_fwd():
         fa.fa_fwd(q, k, v, o, lse, B, Hq, Hkv, N, N, d, scale, 1, None, fa.FA_BF16, None, 0, st)
@@ -279,6 +310,7 @@ def run_device(args):
 
     fwd_ms = timed_launches(call_fwd, args.steps, args.warmup) if do_fwd else [float("nan")]
     dec_ms = timed_launches(call_dec, args.steps, args.warmup) if do_dec else [float("nan")]
+    paged_ms = timed_launches(call_paged, args.steps, args.warmup) if do_paged else [float("nan")]
     if fa.fa_last_device_error(st) != fa.FA_OK:
         raise RuntimeError("device-side timeout recorded during the benchmark")
 
@@ -321,6 +353,7 @@ def run_device(args):
     # ---- reduce over ranks (max time)
     fwd_mean = max_over_ranks(sum(fwd_ms) / len(fwd_ms), dev)
     dec_mean = max_over_ranks(sum(dec_ms) / len(dec_ms), dev)
+    paged_mean = max_over_ranks(sum(paged_ms) / len(paged_ms), dev)
     fwd_e2e_ms = max_over_ranks(fwd_e2e_ms, dev)
     dec_e2e_ms = max_over_ranks(dec_e2e_ms, dev)
     if world > 1:
@@ -341,6 +374,8 @@ def run_device(args):
     tc_peak = peaks["bf16"] if burst else peaks["bf16_sustained"]
     per_launch_tflops = F / (fwd_mean * 1e-3) / 1e12
     per_launch_gbs = kv / (dec_mean * 1e-3) / 1e9
+    pkv = paged_kv_bytes(p_len)
+    paged_gbs = pkv / (paged_mean * 1e-3) / 1e9
     cpu = cpu_baseline_fwd(args.cpu_seconds) if not args.no_cpu else None
     dec_cpu = cpu_baseline_dec(args.cpu_seconds) if not args.no_cpu else None
     line = {
@@ -380,10 +415,20 @@ def run_device(args):
                    "e2e": {"value": round(world * kv / (dec_e2e_ms * 1e-3) / 1e9, 1), "unit": "GB/s",
                            "h2d_bytes_per_step": h2d_dec, "d2h_bytes_per_step": d2h_dec},
                    "cpu_baseline": dec_cpu},
+        "decode_paged": {"value": round(aggregate_rate(pkv, world, paged_mean) / 1e9, 1), "unit": "GB/s",
+                         "ms": round(paged_mean, 4),
+                         "workload": "decode_paged_ragged: B=16, lengths U{1..32768} (seed 1006), Hq=64, Hkv=8, "
+                                     "d=128, 16-token pages in a shuffled pool, split 1024",
+                         "roofline": {"bound": "hbm", "achieved": round(paged_gbs, 1), "peak": peaks["hbm"],
+                                      "unit": "GB/s", "frac": round(paged_gbs / peaks["hbm"], 4),
+                                      "peak_kind": f"measured copy ({peaks['source']})",
+                                      "kernels": "fa_decode_split_kernel<128,paged> (merge in-kernel)",
+                                      "algorithmic_bytes_per_launch": pkv}},
         "e2e": {"value": round(world * F / (fwd_e2e_ms * 1e-3) / 1e12, 2), "unit": "TFLOP/s",
                 "h2d_bytes_per_step": h2d_fwd, "d2h_bytes_per_step": d2h_fwd},
         "cpu_baseline": cpu,
-        "gpu_launches": args.steps * 1 + args.steps * 2,
+        "gpu_launches": args.steps * (int(do_fwd) * 1 + int(do_dec) * 2 + int(do_paged) * 1)
+        + (0 if args.no_e2e else e2e_steps * (int(do_fwd) * 1 + int(do_dec) * 2)),
         "clocks": clocks.summary(),
         "impl": "b200",
     }
@@ -503,7 +548,8 @@ def main():
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--no-cpu", action="store_true", help="skip the CPU oracle baseline")
     ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer end-to-end phases")
-    ap.add_argument("--only", default="all", choices=["all", "fwd", "dec"], help="profiling: run one kernel family")
+    ap.add_argument("--only", default="all", choices=["all", "fwd", "dec", "paged"],
+                    help="profiling: run one kernel family")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
