@@ -49,6 +49,9 @@ class Oracle:
         L.oracle_attention.argtypes = common + [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int]
         L.oracle_attention_rows.argtypes = common + [ctypes.c_void_p, ctypes.c_int64,
                                                      ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int]
+        L.oracle_attention_bwd.argtypes = ([ctypes.c_void_p] * 4 + [ctypes.c_int] * 6 +
+                                           [ctypes.c_double, ctypes.c_int, ctypes.c_void_p] +
+                                           [ctypes.c_void_p] * 3 + [ctypes.c_int])
         L.oracle_hardware_threads.restype = ctypes.c_int
 
     # -- softmax statistics and the merge rule -------------------------------------------
@@ -174,6 +177,30 @@ class Oracle:
         kc = self.gather_pages(k_pages, block_table, seqlens, page_size)
         vc = self.gather_pages(v_pages, block_table, seqlens, page_size)
         return self.decode(q, kc, vc, np.asarray(seqlens), scale, nthreads=nthreads)
+
+    def attention_bwd(self, q, k, v, dout, scale, causal=False, cu_seqlens=None, nthreads=0):
+        """Gradients (dq, dk, dv) of o = attention(q, k, v) for an upstream gradient dout of o
+        (layouts as in attention(); see oracle_attention_bwd in oracle.cpp)."""
+        q, k, v, dout = self._f32(q), self._f32(k), self._f32(v), self._f32(dout)
+        if cu_seqlens is not None:
+            cu = np.ascontiguousarray(cu_seqlens, dtype=np.int32)
+            total, Hq, d = q.shape
+            Hkv = k.shape[1]
+            B, Nq, Nk = len(cu) - 1, total, total
+        else:
+            cu = None
+            B, Nq, Hq, d = q.shape
+            Nk, Hkv = k.shape[1], k.shape[2]
+        dq = np.zeros(q.shape, dtype=np.float64)
+        dk = np.zeros(k.shape, dtype=np.float64)
+        dv = np.zeros(v.shape, dtype=np.float64)
+        rc = self.lib.oracle_attention_bwd(
+            q.ctypes.data, k.ctypes.data, v.ctypes.data, dout.ctypes.data, B, Hq, Hkv, Nq, Nk, d, float(scale),
+            int(bool(causal)), None if cu is None else cu.ctypes.data, dq.ctypes.data, dk.ctypes.data,
+            dv.ctypes.data, int(nthreads))
+        if rc != 0:
+            raise ValueError("oracle_attention_bwd rejected its arguments")
+        return dq, dk, dv
 
     def hardware_threads(self) -> int:
         return int(self.lib.oracle_hardware_threads())

@@ -313,6 +313,104 @@ int oracle_attention_rows(const float* q, const float* k, const float* v, int B,
   return 0;
 }
 
+// Gradients of the attention above with respect to q, k and v, for an upstream gradient dout
+// of o (same layout as o).  "FlashAttention notes", section 5.2 (backward): the backward
+// rebuilds P from q, k and the softmax statistics instead of storing it, then dV = P^T dO and
+// dP = dO V^T; the remaining steps are the derivative of the row softmax.  Here every row is
+// materialised again in fp64 from q, k, v alone (this oracle keeps no forward state):
+//
+//   p_j  = softmax_j(s),  o_i = sum_j p_j v_j                       (as in the forward)
+//   dp_j = <dout_i, v_j>,  D_i = sum_j p_j dp_j  (= <dout_i, o_i>)
+//   ds_j = p_j (dp_j - D_i)                      (softmax derivative)
+//   dq_i  = scale * sum_j ds_j k_j
+//   dk_j += scale * ds_j q_i,   dv_j += p_j dout_i                  (summed over rows and over
+//                                                                  the query heads of the group)
+// Layouts as in oracle_attention (dq like q, dk/dv like k/v); fixed length or varlen.  Threads
+// run over (sequence, key/value head) groups, which own disjoint dk/dv and dq rows.
+int oracle_attention_bwd(const float* q, const float* k, const float* v, const float* dout, int B, int Hq,
+                         int Hkv, int Nq, int Nk, int d, double scale, int causal, const int32_t* cu_seqlens,
+                         double* dq, double* dk, double* dv, int nthreads) {
+  Problem P{q, k, v, B, Hq, Hkv, Nq, Nk, d, scale, causal, cu_seqlens, nullptr};
+  if (check_problem(P) || !dout || !dq || !dk || !dv) return 1;
+  const int G = Hq / Hkv;
+  const int64_t rows_q = cu_seqlens ? (int64_t)Nq : (int64_t)B * Nq;
+  const int64_t rows_k = cu_seqlens ? (int64_t)Nk : (int64_t)B * Nk;
+  for (int64_t t = 0; t < rows_q * Hq * d; ++t) dq[t] = 0.0;
+  for (int64_t t = 0; t < rows_k * Hkv * d; ++t) dk[t] = dv[t] = 0.0;
+  const int64_t units = (int64_t)B * Hkv;
+  parallel_for(units, nthreads, [&](int64_t u, std::vector<double>& scratch) {
+    const int b = (int)(u / Hkv), g = (int)(u % Hkv);
+    std::vector<double> o((size_t)d);
+    for (int hh = 0; hh < G; ++hh) {
+      const int h = g * G + hh;
+      for (int64_t i = 0; i < Nq; ++i) {
+        RowView r = view_row(P, b, h, i);
+        if (!r.valid) break;
+        if (r.jmax <= 0) continue;  // no allowed key: o = 0 and no gradient flows
+        const int64_t n = r.jmax;
+        scratch.resize((size_t)(3 * n));
+        double* s = scratch.data();
+        double* pr = s + n;
+        double* dp = pr + n;
+        for (int64_t j = 0; j < n; ++j) {
+          const float* kj = r.kbase + j * r.kstride;
+          double acc = 0.0;
+          for (int c = 0; c < d; ++c) acc += (double)r.qrow[c] * (double)kj[c];
+          s[j] = P.scale * acc;
+        }
+        double m = kNegInf;
+        for (int64_t j = 0; j < n; ++j) m = std::max(m, s[j]);
+        double l = 0.0;
+        for (int64_t j = 0; j < n; ++j) {
+          pr[j] = std::exp(s[j] - m);
+          l += pr[j];
+        }
+        for (int64_t j = 0; j < n; ++j) pr[j] /= l;
+        const float* dorow = dout + r.orow * d;
+        for (int c = 0; c < d; ++c) o[(size_t)c] = 0.0;
+        for (int64_t j = 0; j < n; ++j) {
+          const float* vj = r.vbase + j * r.kstride;
+          double acc = 0.0;
+          for (int c = 0; c < d; ++c) {
+            o[(size_t)c] += pr[j] * (double)vj[c];
+            acc += (double)dorow[c] * (double)vj[c];
+          }
+          dp[j] = acc;
+        }
+        double D = 0.0;
+        for (int64_t j = 0; j < n; ++j) D += pr[j] * dp[j];
+        double* dqrow = dq + r.orow * d;
+        // dk/dv row of key j: same place in the k/v layout as the key row itself
+        const int64_t kvrow0 = (r.kbase - P.k) / d;  // (k0 * Hkv + g)
+        for (int64_t j = 0; j < n; ++j) {
+#ifdef ORACLE_PLANT_BWD_NO_D
+          const double ds = pr[j] * dp[j];
+#else
+          const double ds = pr[j] * (dp[j] - D);
+#endif
+          const float* kj = r.kbase + j * r.kstride;
+          double* dkj = dk + (kvrow0 + j * Hkv) * d;
+          double* dvj = dv + (kvrow0 + j * Hkv) * d;
+          for (int c = 0; c < d; ++c) {
+#ifdef ORACLE_PLANT_BWD_DQ_NO_SCALE
+            dqrow[c] += ds * (double)kj[c];
+#else
+            dqrow[c] += P.scale * ds * (double)kj[c];
+#endif
+#ifdef ORACLE_PLANT_BWD_DK_FROM_P
+            dkj[c] += P.scale * pr[j] * (double)r.qrow[c];
+#else
+            dkj[c] += P.scale * ds * (double)r.qrow[c];
+#endif
+            dvj[c] += pr[j] * (double)dorow[c];
+          }
+        }
+      }
+    }
+  });
+  return 0;
+}
+
 int oracle_hardware_threads(void) { return (int)std::thread::hardware_concurrency(); }
 
 }  // extern "C"
