@@ -18,8 +18,8 @@ FA_OK, FA_ERR_INVALID_ARG, FA_ERR_UNSUPPORTED, FA_ERR_WORKSPACE, FA_ERR_CUDA, FA
 FA_BF16, FA_F32 = 0, 1
 
 EXPORTED = ("fa_fwd", "fa_fwd_workspace_size", "fa_decode", "fa_decode_workspace_size", "fa_decode_noalloc",
-            "fa_decode_paged", "fa_decode_paged_workspace_size", "fa_last_device_error", "fa_status_string",
-            "fa_device_sm_count")
+            "fa_decode_paged", "fa_decode_paged_workspace_size", "fa_bwd", "fa_bwd_workspace_size",
+            "fa_last_device_error", "fa_status_string", "fa_device_sm_count")
 FA_DECODE_NOALLOC_SCRATCH_BYTES = 16 << 20
 
 
@@ -55,6 +55,10 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
     L.fa_decode_paged.restype = i
     L.fa_decode_paged_workspace_size.argtypes = [i, i, i, i, i, i, i]
     L.fa_decode_paged_workspace_size.restype = sz
+    L.fa_bwd.argtypes = [vp] * 9 + [i] * 6 + [f, i, vp, sz, vp]
+    L.fa_bwd.restype = i
+    L.fa_bwd_workspace_size.argtypes = [i, i, i, i]
+    L.fa_bwd_workspace_size.restype = sz
     L.fa_last_device_error.argtypes = [vp]
     L.fa_last_device_error.restype = i
     L.fa_status_string.argtypes = [i]
@@ -141,6 +145,18 @@ def fa_decode_paged_workspace_size(B, Hq, Hkv, max_pages_per_seq, page_size, d, 
                                                      int(page_size), int(d), int(split_len)))
 
 
+def fa_bwd(q, k, v, o, dout, lse, dq, dk, dv, B, Hq, Hkv, Nq, Nk, d, scale, causal, workspace, workspace_bytes,
+           stream=None) -> None:
+    st = load().fa_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(dout), _ptr(lse), _ptr(dq), _ptr(dk), _ptr(dv),
+                       int(B), int(Hq), int(Hkv), int(Nq), int(Nk), int(d), float(scale), int(bool(causal)),
+                       _ptr(workspace), int(workspace_bytes), _stream(stream))
+    _check(st, "fa_bwd")
+
+
+def fa_bwd_workspace_size(B, Hq, Nq, d) -> int:
+    return int(load().fa_bwd_workspace_size(int(B), int(Hq), int(Nq), int(d)))
+
+
 def fa_last_device_error(stream=None) -> int:
     return int(load().fa_last_device_error(_stream(stream)))
 
@@ -223,3 +239,18 @@ def decode_paged(q, k_pages, v_pages, block_table, seqlens, scale=None, split_le
     fa_decode_paged(q, k_pages, v_pages, block_table, seqlens, out, lse, B, Hq, Hkv, num_pages, page_size, maxp, d,
                     scale, split_len, workspace, ws_bytes, stream)
     return out, lse
+
+
+def backward(q, k, v, o, lse, dout, causal=False, scale=None, workspace=None, stream=None):
+    """dq, dk, dv for q [B,Nq,Hq,d], k/v [B,Nk,Hkv,d], the forward's o and lse, and dout."""
+    import torch
+    B, Nq, Hq, d = q.shape
+    Nk, Hkv = k.shape[1], k.shape[2]
+    if scale is None:
+        scale = d ** -0.5
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    ws_bytes = fa_bwd_workspace_size(B, Hq, Nq, d)
+    if workspace is None:
+        workspace = torch.empty(max(ws_bytes, 1), dtype=torch.uint8, device=q.device)
+    fa_bwd(q, k, v, o, dout, lse, dq, dk, dv, B, Hq, Hkv, Nq, Nk, d, scale, causal, workspace, ws_bytes, stream)
+    return dq, dk, dv

@@ -8,6 +8,7 @@
 #include <mutex>
 
 #include "../../include/fa.h"
+#include "fa_bwd_sm100.cuh"
 #include "fa_decode_sm100.cuh"
 #include "fa_fwd_sm100.cuh"
 
@@ -127,6 +128,32 @@ fa_status launch_decode_paged(const void* kp, const void* vp, const DecParams& p
   if (set_smem(ks, smem) != cudaSuccess) return FA_ERR_CUDA;
   dim3 grid(prm.nsplit, prm.Hkv, prm.B);
   ks<<<grid, kDecThreads, smem, st>>>(mk, mv, prm);
+  return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+}
+
+template <int D>
+fa_status launch_bwd(const void* q, const void* k, const void* v, const BwdParams& prm, cudaStream_t st) {
+  CUtensorMap mq, mk, mv, mdo;
+  const int64_t rows_q = (int64_t)prm.B * prm.Nq, rows_k = (int64_t)prm.B * prm.Nk;
+  if (!make_map(&mq, q, D, prm.Hq, rows_q, kBwdTile) || !make_map(&mdo, prm.dout, D, prm.Hq, rows_q, kBwdTile) ||
+      !make_map(&mk, k, D, prm.Hkv, rows_k, kBwdTile) || !make_map(&mv, v, D, prm.Hkv, rows_k, kBwdTile))
+    return FA_ERR_CUDA;
+  const int sms = sm_count_cached();
+  if (sms <= 0) return FA_ERR_CUDA;
+  const long long pre_rows = (long long)prm.B * prm.Hq * prm.NqPad;
+  const int pre_blocks = (int)std::min<long long>((pre_rows + 7) / 8, (long long)sms * 16);
+  if (pre_blocks > 0) fa_bwd_pre_kernel<D><<<pre_blocks, 256, 0, st>>>(prm);
+  if (cudaGetLastError() != cudaSuccess) return FA_ERR_CUDA;
+  if (prm.Nk > 0) {
+    auto kern = fa_bwd_kernel<D>;
+    const int smem = BwdCfg<D>::kSmemBytes;
+    if (set_smem(kern, smem) != cudaSuccess) return FA_ERR_CUDA;
+    dim3 grid((prm.Nk + kBwdTile - 1) / kBwdTile, prm.Hkv, prm.B);
+    kern<<<grid, kBwdThreads, smem, st>>>(mq, mk, mv, mdo, prm);
+    if (cudaGetLastError() != cudaSuccess) return FA_ERR_CUDA;
+  }
+  const size_t n4 = (size_t)prm.B * prm.Nq * prm.Hq * D / 4;
+  if (n4 > 0) fa_bwd_dq_kernel<D><<<(int)std::min<size_t>((n4 + 255) / 256, (size_t)sms * 8), 256, 0, st>>>(prm);
   return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
 
@@ -336,6 +363,62 @@ fa_status fa_decode_paged(const void* q, const void* k_pages, const void* v_page
                  : launch_decode_paged<128>(k_pages, v_pages, prm, st);
 }
 
+size_t fa_bwd_workspace_size(int B, int Hq, int Nq, int d) {
+  if (B <= 0 || Hq <= 0 || Nq <= 0 || d <= 0) return 0;
+  const size_t pad = (size_t)(Nq + kBwdTile - 1) / kBwdTile * kBwdTile;
+  return 2 * align_up((size_t)B * Hq * pad * 4, 256) + align_up((size_t)B * Nq * Hq * d * 4, 256);
+}
+
+fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, const void* dout, const float* lse,
+                 void* dq, void* dk, void* dv, int B, int Hq, int Hkv, int Nq, int Nk, int d, float scale, int causal,
+                 void* workspace, size_t workspace_bytes, void* stream) {
+  if (!q || !k || !v || !o || !dout || !lse || !dq || !dk || !dv) return FA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(dout) || !aligned16(dq) ||
+      !aligned16(dk) || !aligned16(dv) || (reinterpret_cast<uintptr_t>(lse) & 3u) != 0)
+    return FA_ERR_INVALID_ARG;
+  if (B < 0 || Hq <= 0 || Hkv <= 0 || Nq < 0 || Nk < 0) return FA_ERR_INVALID_ARG;
+  if (!(scale > 0.f) || !std::isfinite(scale)) return FA_ERR_INVALID_ARG;
+  if (Hq % Hkv != 0) return FA_ERR_UNSUPPORTED;
+  if (d != 64 && d != 128) return FA_ERR_UNSUPPORTED;
+  const int64_t rows_q = (int64_t)B * Nq, rows_k = (int64_t)B * Nk;
+  if (rows_q >= (int64_t(1) << 31) || rows_k >= (int64_t(1) << 31)) return FA_ERR_UNSUPPORTED;
+  if (B > 65535 || Hkv > 65535) return FA_ERR_UNSUPPORTED;
+  if (B == 0 || (Nq == 0 && Nk == 0)) return FA_OK;
+  const size_t need = fa_bwd_workspace_size(B, Hq, Nq, d);
+  if (need > 0 && (!workspace || workspace_bytes < need || !aligned16(workspace))) return FA_ERR_WORKSPACE;
+  BwdParams prm{};
+  const int pad = (Nq + kBwdTile - 1) / kBwdTile * kBwdTile;
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  prm.lse2 = reinterpret_cast<float*>(ws);
+  prm.dvec = reinterpret_cast<float*>(ws + align_up((size_t)B * Hq * pad * 4, 256));
+  prm.dq_acc = reinterpret_cast<float*>(ws + 2 * align_up((size_t)B * Hq * pad * 4, 256));
+  prm.o = static_cast<const __nv_bfloat16*>(o);
+  prm.dout = static_cast<const __nv_bfloat16*>(dout);
+  prm.lse = lse;
+  prm.dq = static_cast<__nv_bfloat16*>(dq);
+  prm.dk = static_cast<__nv_bfloat16*>(dk);
+  prm.dv = static_cast<__nv_bfloat16*>(dv);
+  prm.B = B;
+  prm.Hq = Hq;
+  prm.Hkv = Hkv;
+  prm.G = Hq / Hkv;
+  prm.Nq = Nq;
+  prm.Nk = Nk;
+  prm.NqPad = pad;
+  prm.causal = causal ? 1 : 0;
+  prm.scale = scale;
+  prm.tau = (float)((double)scale * 1.4426950408889634074);
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (Nq == 0) {
+    // no query: every gradient is zero
+    if (cudaMemsetAsync(dk, 0, (size_t)rows_k * Hkv * d * 2, st) != cudaSuccess ||
+        cudaMemsetAsync(dv, 0, (size_t)rows_k * Hkv * d * 2, st) != cudaSuccess)
+      return FA_ERR_CUDA;
+    return FA_OK;
+  }
+  return d == 64 ? launch_bwd<64>(q, k, v, prm, st) : launch_bwd<128>(q, k, v, prm, st);
+}
+
 fa_status fa_last_device_error(void* stream) {
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   if (cudaStreamSynchronize(st) != cudaSuccess) return FA_ERR_CUDA;
@@ -344,7 +427,9 @@ fa_status fa_last_device_error(void* stream) {
   if (w != 0) {
     const unsigned int zero = 0;
     if (cudaMemcpyToSymbol(g_error_word, &zero, sizeof(zero)) != cudaSuccess) return FA_ERR_CUDA;
-    return (w & kErrTimeout) ? FA_ERR_TIMEOUT : FA_ERR_INVALID_ARG;
+    if (w & kErrTimeout) return FA_ERR_TIMEOUT;
+    if (w & kErrSmem) return FA_ERR_CUDA;
+    return FA_ERR_INVALID_ARG;
   }
   return FA_OK;
 }

@@ -1,0 +1,428 @@
+// Backward attention kernels for sm_100a.
+//
+// The method ("FlashAttention notes", section 5.2, backward; "LLM basics: from Attention to
+// FlashAttention", chapter 3 section 6): the N x N matrices are not kept from the forward.
+// The backward rebuilds P tile by tile from Q, K and the saved per-row logsumexp,
+//   P = exp(scale * Q K^T - lse),
+// and forms the gradients with it on chip:
+//   dV = P^T dO,  dP = dO V^T,  dS = P o (dP - D)  with  D_i = sum_c dO_ic O_ic,
+//   dQ = scale * dS K,  dK = scale * dS^T Q.
+// Only dQ, dK and dV (and two vectors per row) reach device memory.
+//
+// Three launches:
+//   fa_bwd_pre_kernel   D_i and lse_i * log2(e) per query row (padded to whole tiles, with
+//                       +inf where no key is allowed so that P = 0 there), and zeroes the
+//                       fp32 dQ accumulator.
+//   fa_bwd_kernel       one CTA per (128-key tile, K/V head, sequence): K and V stay in
+//                       shared memory while (query head of the group, 128-query tile) pairs
+//                       stream past; dK and dV accumulate in TMEM over all of them (the group
+//                       sum of GQA included), dQ of each pair is added to the fp32 accumulator
+//                       with vector reductions.
+//   fa_bwd_dq_kernel    dQ = scale * accumulator, rounded to bf16.
+//
+// B200 mapping of fa_bwd_kernel (384 threads, one CTA per SM):
+//   warp 0      TMA producer (K, V once; Q, dO and the row vectors per pair, double-buffered)
+//   warp 1      tcgen05.mma issuer and TMEM owner
+//   warps 2-3   idle
+//   warps 4-11  two elementwise warpgroups; thread = key row = TMEM lane, warpgroup w takes
+//               query columns 64w..64w+63 of each pair, then dQ columns of its half.
+// Per pair, with the key tile as the M side (TMEM lanes = keys):
+//   S^T = K Q^T -> TMEM[0,128)      dP^T = V dO^T -> TMEM[128,256)       (tcgen05, SS)
+//   P^T = 2^(S^T tau - lse2), dS^T = P^T o (dP^T - D)                    (elementwise)
+//   P^T (bf16) over TMEM[0,64), dS^T (bf16) over TMEM[128,192), dS^T also to shared memory
+//   dV += P^T dO,  dK += dS^T Q               (tcgen05, A from TMEM; TMEM[256,256+2d))
+//   dQ = dS K -> TMEM[64,128) and TMEM[192,256) (two 64-column halves; A = dS from shared
+//   memory, query-major)
+// Every operand tile is stored once (128 rows, 64-column panels, 128-byte swizzle) and read
+// either K-major or MN-major through its descriptor.
+#pragma once
+
+#include "fa_device.cuh"
+
+namespace fa {
+
+struct BwdParams {
+  const __nv_bfloat16* o;     // [B, Nq, Hq, D]
+  const __nv_bfloat16* dout;  // [B, Nq, Hq, D]
+  const float* lse;           // [B, Hq, Nq] (natural log)
+  float* lse2;                // [B, Hq, NqPad] lse * log2(e); +inf where P must be 0
+  float* dvec;                // [B, Hq, NqPad] D_i = sum_c dO_ic O_ic
+  float* dq_acc;              // [B, Nq, Hq, D] fp32
+  __nv_bfloat16* dq;          // [B, Nq, Hq, D]
+  __nv_bfloat16* dk;          // [B, Nk, Hkv, D]
+  __nv_bfloat16* dv;          // [B, Nk, Hkv, D]
+  int B, Hq, Hkv, G, Nq, Nk, NqPad;
+  int causal;
+  float tau;    // scale * log2(e)
+  float scale;
+};
+
+constexpr int kBwdThreads = 384;
+constexpr int kBwdTile = 128;            // keys per CTA tile and queries per pair
+constexpr unsigned int kErrSmem = 4u;    // the kernel's shared-memory carve did not fit
+constexpr int kBwdMaxSmem = 232448;      // sm_100 per-block limit
+
+template <int D>
+struct BwdCfg {
+  static constexpr int kTileBytes = kBwdTile * D * 2;
+  static constexpr int kChunkBytes = kBwdTile * 128;  // 128 rows x one 64-column panel
+  static constexpr int kVecBytes = kBwdTile * 4;
+  static constexpr int kOffK = 0;
+  static constexpr int kOffV = kTileBytes;
+  static constexpr int kOffQ = 2 * kTileBytes;   // [2]
+  static constexpr int kOffDO = 4 * kTileBytes;  // [2]
+  static constexpr int kOffDS = 6 * kTileBytes;  // 128 keys x 128 queries bf16
+  static constexpr int kOffVec = kOffDS + kBwdTile * kBwdTile * 2;  // [slot][lse2, D]
+  static constexpr int kOffBar = kOffVec + 4 * kVecBytes;
+  static constexpr int kNumBars = 16;
+  static constexpr int kUsed = kOffBar + kNumBars * 8 + 16;
+  static constexpr int kSmemBytes = (kUsed + 1024 < kBwdMaxSmem) ? kUsed + 1024 : kBwdMaxSmem;
+  // TMEM columns
+  static constexpr uint32_t kColS = 0, kColDP = 128, kColDV = 256, kColDK = 256 + D;
+};
+
+// ------------------------------------------------------------------ pre: D and lse2, zero dQ
+template <int D>
+__global__ void __launch_bounds__(256) fa_bwd_pre_kernel(const BwdParams p) {
+  const int warps = blockDim.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const long long rows = (long long)p.B * p.Hq * p.NqPad;
+  constexpr int E = D / 32;  // elements per lane
+  for (long long w = (long long)blockIdx.x * warps + (threadIdx.x >> 5); w < rows; w += (long long)gridDim.x * warps) {
+    const int q = (int)(w % p.NqPad);
+    const long long bh = w / p.NqPad;
+    const int h = (int)(bh % p.Hq), b = (int)(bh / p.Hq);
+    float dsum = 0.f, l2 = INFINITY;
+    if (q < p.Nq) {
+      const size_t row = ((size_t)b * p.Nq + q) * p.Hq + h;
+      const __nv_bfloat16* orow = p.o + row * D + lane * E;
+      const __nv_bfloat16* drow = p.dout + row * D + lane * E;
+#pragma unroll
+      for (int e = 0; e < E; e += 2) {
+        const float2 a = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(orow + e));
+        const float2 g = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(drow + e));
+        dsum = fmaf(a.x, g.x, fmaf(a.y, g.y, dsum));
+      }
+      float* acc = p.dq_acc + row * D + lane * E;
+#pragma unroll
+      for (int e = 0; e < E; ++e) acc[e] = 0.f;
+      const float l = p.lse[((size_t)b * p.Hq + h) * p.Nq + q];
+      l2 = (l == -INFINITY) ? INFINITY : l * 1.4426950408889634f;
+    }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) dsum += __shfl_xor_sync(0xffffffffu, dsum, off);
+    if (lane == 0) {
+      p.dvec[w] = dsum;
+      p.lse2[w] = l2;
+    }
+  }
+}
+
+// ------------------------------------------------------------------ post: dQ to bf16
+template <int D>
+__global__ void __launch_bounds__(256) fa_bwd_dq_kernel(const BwdParams p) {
+  const size_t n4 = (size_t)p.B * p.Nq * p.Hq * D / 4;
+  const size_t stride = (size_t)gridDim.x * blockDim.x;
+  for (size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x; i < n4; i += stride) {
+    const float4 x = reinterpret_cast<const float4*>(p.dq_acc)[i];
+    uint2 w;
+    w.x = pack_bf16x2(x.x * p.scale, x.y * p.scale);
+    w.y = pack_bf16x2(x.z * p.scale, x.w * p.scale);
+    reinterpret_cast<uint2*>(p.dq)[i] = w;
+  }
+}
+
+// ------------------------------------------------------------------ main
+template <int D>
+__global__ void __launch_bounds__(kBwdThreads, 1)
+    fa_bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                  const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmDO,
+                  const BwdParams p) {
+  using C = BwdCfg<D>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  {
+    uint32_t dyn;
+    asm volatile("mov.u32 %0, %%dynamic_smem_size;" : "=r"(dyn));
+    if ((uint32_t)(smem - smem_raw) + (uint32_t)C::kUsed > dyn) {
+      if (threadIdx.x == 0) atomicOr(&g_error_word, kErrSmem);
+      return;
+    }
+  }
+  uint8_t* sK = smem + C::kOffK;
+  uint8_t* sV = smem + C::kOffV;
+  uint8_t* sQ = smem + C::kOffQ;
+  uint8_t* sDO = smem + C::kOffDO;
+  uint8_t* sDS = smem + C::kOffDS;
+  float* sVec = reinterpret_cast<float*>(smem + C::kOffVec);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kOffBar);
+  uint64_t* kv_full = bars + 0;
+  uint64_t* q_full = bars + 1;     // [2]
+  uint64_t* q_empty = bars + 3;    // [2]
+  uint64_t* sdp_full = bars + 5;   // S^T and dP^T in TMEM
+  uint64_t* ld_done = bars + 6;    // both warpgroups have read S^T and dP^T
+  uint64_t* pds_ready = bars + 7;  // P^T, dS^T in TMEM and dS in shared memory
+  uint64_t* dq_full = bars + 8;    // dQ in TMEM
+  uint64_t* dq_free = bars + 9;    // dQ read out
+  uint64_t* acc_done = bars + 10;  // last dK/dV product complete
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + C::kNumBars);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int ntile = blockIdx.x, kvh = blockIdx.y, b = blockIdx.z;
+  const int n0 = ntile * kBwdTile;
+  const int diag = p.Nk - p.Nq;  // causal: key j is allowed for query i iff j <= i + diag
+  const int nq_tiles = (p.Nq + kBwdTile - 1) / kBwdTile;
+  int i_lo = 0;
+  if (p.causal) {
+    const int need = n0 - diag - (kBwdTile - 1);  // first tile whose last query sees key n0
+    i_lo = need <= 0 ? 0 : (need + kBwdTile - 1) / kBwdTile;
+  }
+  const int ntq = max(0, nq_tiles - i_lo);
+  const int T = ntq * p.G;  // (query head, query tile) pairs; heads outer
+
+  if (threadIdx.x == 0) {
+    mbar_init(kv_full, 1);
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(q_full + s, 1);
+      mbar_init(q_empty + s, 1);
+    }
+    mbar_init(sdp_full, 1);
+    mbar_init(ld_done, 8);
+    mbar_init(pds_ready, 8);
+    mbar_init(dq_full, 1);
+    mbar_init(dq_free, 8);
+    mbar_init(acc_done, 1);
+    fence_barrier_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0) {
+    // ============================================================ TMA producer
+    if (T > 0) {
+      mbar_arrive_expect_tx_elect(kv_full, 2 * C::kTileBytes);
+      for (int c = 0; c < D / 64; ++c) {
+        tma_load_3d_elect(sK + c * C::kChunkBytes, &tmK, c * 64, kvh, b * p.Nk + n0, kv_full);
+        tma_load_3d_elect(sV + c * C::kChunkBytes, &tmV, c * 64, kvh, b * p.Nk + n0, kv_full);
+      }
+      for (int t = 0; t < T; ++t) {
+        const int slot = t & 1;
+        if (t >= 2 && !warp_wait(q_empty + slot, ((t >> 1) - 1) & 1)) break;
+        const int h = kvh * p.G + t / ntq;
+        const int q0 = (i_lo + t % ntq) * kBwdTile;
+        mbar_arrive_expect_tx_elect(q_full + slot, 2 * C::kTileBytes + 2 * C::kVecBytes);
+        for (int c = 0; c < D / 64; ++c) {
+          tma_load_3d_elect(sQ + slot * C::kTileBytes + c * C::kChunkBytes, &tmQ, c * 64, h, b * p.Nq + q0,
+                            q_full + slot);
+          tma_load_3d_elect(sDO + slot * C::kTileBytes + c * C::kChunkBytes, &tmDO, c * 64, h, b * p.Nq + q0,
+                            q_full + slot);
+        }
+        const size_t voff = ((size_t)b * p.Hq + h) * p.NqPad + q0;
+        bulk_load_elect(sVec + (slot * 2 + 0) * kBwdTile, p.lse2 + voff, C::kVecBytes, q_full + slot);
+        bulk_load_elect(sVec + (slot * 2 + 1) * kBwdTile, p.dvec + voff, C::kVecBytes, q_full + slot);
+      }
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    // ============================================================ MMA issuer
+    if (T > 0) {
+      constexpr uint32_t idS = idesc_bf16_f32(kBwdTile, kBwdTile, false);  // K-major A and B
+      constexpr uint32_t idAcc = idesc_bf16_f32(kBwdTile, D, true);        // B MN-major
+      constexpr uint32_t idQ = idesc_bf16_f32_mn(kBwdTile, 64, true, true);
+      const uint32_t kb = smem_u32(sK), vb = smem_u32(sV), qb = smem_u32(sQ), dob = smem_u32(sDO);
+      const uint32_t dsb = smem_u32(sDS);
+      bool ok = warp_wait(kv_full, 0);
+      tc_fence_after();
+      for (int t = 0; t < T && ok; ++t) {
+        const int slot = t & 1;
+        if (!warp_wait(q_full + slot, (t >> 1) & 1)) break;
+        if (t > 0 && !warp_wait(dq_free, (t - 1) & 1)) break;
+        tc_fence_after();
+        const uint32_t qs = qb + slot * C::kTileBytes, ds = dob + slot * C::kTileBytes;
+        // S^T = K Q^T and dP^T = V dO^T (k-steps of 16 along d)
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = (kk >> 2) * C::kChunkBytes + (kk & 3) * 32;
+          umma_ss_elect(tmem + C::kColS, smem_desc_sw128(kb + off, 16, 1024), smem_desc_sw128(qs + off, 16, 1024),
+                        idS, kk > 0 ? 1u : 0u);
+        }
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = (kk >> 2) * C::kChunkBytes + (kk & 3) * 32;
+          umma_ss_elect(tmem + C::kColDP, smem_desc_sw128(vb + off, 16, 1024), smem_desc_sw128(ds + off, 16, 1024),
+                        idS, kk > 0 ? 1u : 0u);
+        }
+        umma_commit_elect(sdp_full);
+        if (!warp_wait(pds_ready, t & 1)) break;
+        tc_fence_after();
+        // dV += P^T dO, dK += dS^T Q (k-steps of 16 queries; A from TMEM)
+#pragma unroll
+        for (int kk = 0; kk < kBwdTile / 16; ++kk) {
+          const uint32_t acc = (t > 0 || kk > 0) ? 1u : 0u;
+          umma_ts_elect(tmem + C::kColDV, tmem + C::kColS + kk * 8,
+                        smem_desc_sw128(ds + kk * 16 * 128, C::kChunkBytes, 1024), idAcc, acc);
+          umma_ts_elect(tmem + C::kColDK, tmem + C::kColDP + kk * 8,
+                        smem_desc_sw128(qs + kk * 16 * 128, C::kChunkBytes, 1024), idAcc, acc);
+        }
+        // dQ = dS K in 64-column halves (k-steps of 16 keys; A query-major from shared memory)
+#pragma unroll
+        for (int hh = 0; hh < D / 64; ++hh) {
+#pragma unroll
+          for (int kk = 0; kk < kBwdTile / 16; ++kk)
+            umma_ss_elect(tmem + (hh ? C::kColDP : C::kColS) + 64,
+                          smem_desc_sw128(dsb + kk * 16 * 128, C::kChunkBytes, 1024),
+                          smem_desc_sw128(kb + hh * C::kChunkBytes + kk * 16 * 128, C::kChunkBytes, 1024), idQ,
+                          kk > 0 ? 1u : 0u);
+        }
+        umma_commit_elect(dq_full);
+        umma_commit_elect(q_empty + slot);
+      }
+      umma_commit_elect(acc_done);
+    }
+    __syncwarp();
+  } else if (warp >= 4) {
+    // ============================================================ elementwise warpgroups
+    const int wg = (warp - 4) >> 2;
+    const int r = (warp & 3) * 32 + lane;  // key row of the tile = TMEM lane
+    const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
+    const int key = n0 + r;
+    const bool key_ok = key < p.Nk;
+    const float tau = p.tau;
+    bool ok = true;
+    for (int t = 0; t < T && ok; ++t) {
+      const int slot = t & 1;
+      const int h = kvh * p.G + t / ntq;
+      const int q0 = (i_lo + t % ntq) * kBwdTile;
+      if (!warp_wait(q_full + slot, (t >> 1) & 1) || !warp_wait(sdp_full, t & 1)) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      const float* l2 = sVec + (slot * 2 + 0) * kBwdTile + 64 * wg;
+      const float* dd = sVec + (slot * 2 + 1) * kBwdTile + 64 * wg;
+      uint32_t pk[32], dsk[32];
+#pragma unroll
+      for (int c = 0; c < 2; ++c) {
+        uint32_t sv[32], dpv[32];
+        tmem_ld32(tmem + lane_off + C::kColS + 64 * wg + 32 * c, sv);
+        tmem_ld32(tmem + lane_off + C::kColDP + 64 * wg + 32 * c, dpv);
+        tmem_wait_ld();
+        // allowed iff key_ok and (not causal or key <= q + diag), q = q0 + 64 wg + 32 c + e
+        const int qfirst = q0 + 64 * wg + 32 * c;
+        int lim = 0;  // columns e < lim are masked
+        if (!key_ok) lim = 32;
+        else if (p.causal) lim = min(32, max(0, key - diag - qfirst));
+#pragma unroll
+        for (int e = 0; e < 16; ++e) {
+          const float4 lv = *reinterpret_cast<const float4*>(l2 + 32 * c + 4 * (e >> 1));
+          const float4 dv4 = *reinterpret_cast<const float4*>(dd + 32 * c + 4 * (e >> 1));
+          const float la = (e & 1) ? lv.z : lv.x, lb = (e & 1) ? lv.w : lv.y;
+          const float da = (e & 1) ? dv4.z : dv4.x, db = (e & 1) ? dv4.w : dv4.y;
+          float p0 = ex2_approx(fmaf(__uint_as_float(sv[2 * e]), tau, -la));
+          float p1 = ex2_approx(fmaf(__uint_as_float(sv[2 * e + 1]), tau, -lb));
+          if (2 * e < lim) p0 = 0.f;
+          if (2 * e + 1 < lim) p1 = 0.f;
+          const float ds0 = p0 * (__uint_as_float(dpv[2 * e]) - da);
+          const float ds1 = p1 * (__uint_as_float(dpv[2 * e + 1]) - db);
+          pk[16 * c + e] = pack_bf16x2(p0, p1);
+          dsk[16 * c + e] = pack_bf16x2(ds0, ds1);
+        }
+      }
+      // dS row r (queries 64 wg .. 64 wg + 63) into the query-major A tile: panel wg, row r,
+      // 16-byte unit u stored at u ^ (r % 8) (128-byte swizzle)
+      {
+        uint8_t* row = sDS + wg * C::kChunkBytes + r * 128;
+#pragma unroll
+        for (int u = 0; u < 8; ++u)
+          *reinterpret_cast<uint4*>(row + ((u ^ (r & 7)) << 4)) =
+              make_uint4(dsk[4 * u], dsk[4 * u + 1], dsk[4 * u + 2], dsk[4 * u + 3]);
+      }
+      // P^T and dS^T go over the first 64 columns of their regions, which the other
+      // warpgroup may still be reading: wait until both have read S^T and dP^T
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(ld_done);
+      if (!warp_wait(ld_done, t & 1)) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      tmem_st32(tmem + lane_off + C::kColS + 32 * wg, pk);
+      tmem_st32(tmem + lane_off + C::kColDP + 32 * wg, dsk);
+      tmem_wait_st();
+      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");  // dS tile -> tensor core
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(pds_ready);
+      // dQ of this pair: TMEM lane r = query q0 + r; this warpgroup adds its half of d
+      if (!warp_wait(dq_full, t & 1)) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      {
+        constexpr int kCols = D / 2;  // columns of d per warpgroup
+        const uint32_t src = (D == 128) ? (tmem + lane_off + (wg ? C::kColDP : C::kColS) + 64)
+                                        : (tmem + lane_off + C::kColS + 64 + 32 * wg);
+        const int q = q0 + r;
+        float* dst = p.dq_acc + (((size_t)b * p.Nq + q) * p.Hq + h) * D + wg * kCols;
+#pragma unroll
+        for (int c = 0; c < kCols / 32; ++c) {
+          uint32_t a[32];
+          tmem_ld32(src + 32 * c, a);
+          tmem_wait_ld();
+          if (q < p.Nq) {
+#pragma unroll
+            for (int e = 0; e < 32; e += 4)
+              red_add_v4(dst + 32 * c + e, __uint_as_float(a[e]), __uint_as_float(a[e + 1]),
+                         __uint_as_float(a[e + 2]), __uint_as_float(a[e + 3]));
+          }
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(dq_free);
+    }
+    // ---- epilogue: dV (warpgroup 0) and dK = scale * acc (warpgroup 1), rows of this key tile
+    // (T is uniform over the CTA, so every warp takes the same path to the collective loads)
+    const bool have = T > 0 && ok && warp_wait(acc_done, 0);
+    tc_fence_after();
+    __nv_bfloat16* dst = (wg ? p.dk : p.dv) + (((size_t)b * p.Nk + key) * p.Hkv + kvh) * D;
+    const float mul = wg ? p.scale : 1.f;
+#pragma unroll
+    for (int c = 0; c < D / 32; ++c) {
+      uint32_t a[32];
+      if (have) {
+        tmem_ld32(tmem + lane_off + (wg ? C::kColDK : C::kColDV) + 32 * c, a);
+        tmem_wait_ld();
+      } else {
+#pragma unroll
+        for (int e = 0; e < 32; ++e) a[e] = 0u;
+      }
+      if (key_ok) {
+        uint4* d4 = reinterpret_cast<uint4*>(dst + 32 * c);
+#pragma unroll
+        for (int e = 0; e < 4; ++e)
+          d4[e] = make_uint4(pack_bf16x2(__uint_as_float(a[8 * e]) * mul, __uint_as_float(a[8 * e + 1]) * mul),
+                             pack_bf16x2(__uint_as_float(a[8 * e + 2]) * mul, __uint_as_float(a[8 * e + 3]) * mul),
+                             pack_bf16x2(__uint_as_float(a[8 * e + 4]) * mul, __uint_as_float(a[8 * e + 5]) * mul),
+                             pack_bf16x2(__uint_as_float(a[8 * e + 6]) * mul, __uint_as_float(a[8 * e + 7]) * mul));
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+}  // namespace fa

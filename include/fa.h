@@ -14,6 +14,7 @@
  *              results are merged with the same m/l rule ("FlashAttention-3 (FA-3)",
  *              section 4 "FlashDecoding"; "FlashAttention notes", section 4).
  *   fa_decode_paged  the same decode over a paged cache addressed through a block table.
+ *   fa_bwd     the backward of fa_fwd by recomputation from the saved logsumexp.
  *
  * Conventions for every entry point:
  *   - All tensor pointers are DEVICE pointers owned by the caller.  The library never
@@ -82,6 +83,25 @@ FA_EXPORT fa_status fa_fwd(const void* q, const void* k, const void* v, void* o,
                  void* workspace, size_t workspace_bytes, void* stream);
 
 FA_EXPORT size_t fa_fwd_workspace_size(int B, int Hq, int Hkv, int Nq, int Nk, int d, fa_dtype in_dtype, int varlen);
+
+/* Backward of fa_fwd (fixed length): gradients dq, dk, dv of o = attention(q, k, v) for an
+ * upstream gradient dout of o ("FlashAttention notes", section 5.2 backward: P is rebuilt on
+ * chip from q, k and the saved logsumexp instead of being stored; dV = P^T dO, dP = dO V^T,
+ * dS = P o (dP - D) with D_i = sum_c dO_ic O_ic, dQ = scale dS K, dK = scale dS^T Q).
+ *
+ * q, o, dout, dq [B, Nq, Hq, d] bf16; k, v, dk, dv [B, Nk, Hkv, d] bf16; lse [B, Hq, Nq] fp32,
+ * the natural-log logsumexp that fa_fwd wrote for (q, k, v, scale, causal), and o the output
+ * it wrote.  Same scale, causal rule and head grouping as fa_fwd; dk and dv sum over the
+ * query heads of each group.  Accumulation is fp32; P and dS are rounded to bf16 for the
+ * tensor-core products; dq, dk, dv are rounded to bf16 (nearest even).
+ * d 64 or 128; pointers 16-byte aligned (lse 4-byte aligned).
+ * workspace: at least fa_bwd_workspace_size(B, Hq, Nq, d) bytes (two padded fp32 row vectors
+ * and an fp32 dq accumulator); its contents need not be initialised. */
+FA_EXPORT fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, const void* dout,
+                           const float* lse, void* dq, void* dk, void* dv, int B, int Hq, int Hkv, int Nq, int Nk,
+                           int d, float scale, int causal, void* workspace, size_t workspace_bytes, void* stream);
+
+FA_EXPORT size_t fa_bwd_workspace_size(int B, int Hq, int Nq, int d);
 
 /* Split-KV decode: one query token per sequence against its KV cache.
  *
@@ -162,9 +182,10 @@ FA_EXPORT size_t fa_decode_paged_workspace_size(int B, int Hq, int Hkv, int max_
                                                 int split_len);
 
 /* Waits for `stream`, then returns FA_ERR_TIMEOUT if any kernel of this library recorded a
- * device-side timeout since the previous call, else FA_ERR_INVALID_ARG if a kernel recorded
- * an invalid device-side input (a block-table entry out of range), and clears the record;
- * FA_ERR_CUDA if the stream reports an error; else FA_OK. */
+ * device-side timeout since the previous call, else FA_ERR_CUDA if a kernel found its shared
+ * memory carve-out too small, else FA_ERR_INVALID_ARG if a kernel recorded an invalid
+ * device-side input (a block-table entry out of range), and clears the record; FA_ERR_CUDA
+ * if the stream reports an error; else FA_OK. */
 FA_EXPORT fa_status fa_last_device_error(void* stream);
 
 /* Static description of a status code. */

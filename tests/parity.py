@@ -60,3 +60,32 @@ def check_lse(l_gpu: np.ndarray, l_ref: np.ndarray, what: str = "lse") -> float:
     m = float(err.max()) if err.size else 0.0
     assert m <= LSE_ABS, f"{what}: max lse error {m}"
     return m
+
+
+# Gradients (backward).  No tolerance is stated for them; this one follows from the
+# arithmetic: P and dS are rounded to bf16 (relative 2^-9) before the tensor-core products
+# and every gradient is rounded to bf16 on output, so each element may carry a few bf16
+# rounding errors of the terms it sums.  Bound: the relative Frobenius error of each tensor
+# at most 1e-2, and every element within 2e-2 of the tensor's largest reference magnitude.
+GRAD_REL_FRO = 1e-2
+GRAD_MAX_REL = 2e-2
+GRAD_ZERO_ABS = 1e-4
+
+
+def check_grad(g_gpu: np.ndarray, g_ref: np.ndarray, what: str) -> dict:
+    assert g_gpu.shape == g_ref.shape, (g_gpu.shape, g_ref.shape)
+    assert np.all(np.isfinite(g_gpu)), f"{what}: non-finite gradient"
+    err = np.abs(g_gpu - g_ref)
+    scale = float(np.abs(g_ref).max()) if g_ref.size else 0.0
+    fro = float(np.linalg.norm(g_ref))
+    stats = {"rel_fro": float(np.linalg.norm(err)) / fro if fro > 0 else float(np.linalg.norm(err)),
+             "max_rel": float(err.max()) / scale if scale > 0 else float(err.max()) if err.size else 0.0}
+    if fro == 0.0:
+        # an exactly-zero gradient (e.g. dQ with a single key: dP - D cancels) comes out of the
+        # fp32 arithmetic as rounding noise of the cancelled terms, which are O(1) for N(0,1)
+        # inputs
+        assert float(np.abs(g_gpu).max()) <= GRAD_ZERO_ABS, f"{what}: reference is zero, gpu is {stats}"
+        return stats
+    assert stats["rel_fro"] <= GRAD_REL_FRO, f"{what}: relative Frobenius error {stats}"
+    assert stats["max_rel"] <= GRAD_MAX_REL, f"{what}: largest element error {stats}"
+    return stats
