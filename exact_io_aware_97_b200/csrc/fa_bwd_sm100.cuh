@@ -372,22 +372,28 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                                         : (tmem + lane_off + C::kColS + 64 + 32 * wg);
         const int q = q0 + r;
         float* dst = p.dq_acc + (((size_t)b * p.Nq + q) * p.Hq + h) * D + wg * kCols;
+        uint32_t a0[32], a1[32];
+        tmem_ld32(src, a0);
+        if (kCols == 64) tmem_ld32(src + 32, a1);
+        tmem_wait_ld();
+        // TMEM is free again as soon as the values are in registers: release it before the
+        // reductions, so the next pair's products start while they drain
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(dq_free);
+        if (q < p.Nq) {
 #pragma unroll
-        for (int c = 0; c < kCols / 32; ++c) {
-          uint32_t a[32];
-          tmem_ld32(src + 32 * c, a);
-          tmem_wait_ld();
-          if (q < p.Nq) {
+          for (int e = 0; e < 32; e += 4)
+            red_add_v4(dst + e, __uint_as_float(a0[e]), __uint_as_float(a0[e + 1]), __uint_as_float(a0[e + 2]),
+                       __uint_as_float(a0[e + 3]));
+          if (kCols == 64) {
 #pragma unroll
             for (int e = 0; e < 32; e += 4)
-              red_add_v4(dst + 32 * c + e, __uint_as_float(a[e]), __uint_as_float(a[e + 1]),
-                         __uint_as_float(a[e + 2]), __uint_as_float(a[e + 3]));
+              red_add_v4(dst + 32 + e, __uint_as_float(a1[e]), __uint_as_float(a1[e + 1]),
+                         __uint_as_float(a1[e + 2]), __uint_as_float(a1[e + 3]));
           }
         }
       }
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(dq_free);
     }
     // ---- epilogue: dV (warpgroup 0) and dK = scale * acc (warpgroup 1), rows of this key tile
     // (T is uniform over the CTA, so every warp takes the same path to the collective loads)
