@@ -45,6 +45,7 @@ FALLBACK_BF16_TFLOPS = 1590.0
 FWD = si.WORKLOADS["gqa_causal_8k"]
 DEC = si.WORKLOADS["decode_split_kv"]
 PAGED = si.WORKLOADS["decode_paged_ragged"]
+DOUT_ID = 9  # stream id of the backward's upstream gradient
 
 
 def fwd_flops(w=FWD) -> float:
@@ -240,7 +241,14 @@ def run_device(args):
     do_fwd = args.only in ("all", "fwd")
     do_dec = args.only in ("all", "dec")
     do_paged = args.only in ("all", "paged")
-    if not do_fwd:
+    do_bwd = args.only in ("all", "bwd")
+    if do_bwd:
+        h_do_f = torch.from_numpy(inputs("fwd", seed, DOUT_ID, (B, N, Hq, d))).to(torch.bfloat16)
+        b_do = h_do_f.to(dev)
+        b_dq, b_dk, b_dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+        b_ws_bytes = fa.fa_bwd_workspace_size(B, Hq, N, d)
+        b_ws = torch.empty(b_ws_bytes, dtype=torch.uint8, device=dev)
+    if not do_fwd and not do_bwd:
         del q, k, v, o, lse
     wd = DEC
     dseed = replica_seed(wd["seed"], rank)
@@ -275,6 +283,9 @@ def run_device(args):
     p_lse = torch.empty((pB, pHq), dtype=torch.float32, device=dev)
     p_ws_bytes = fa.fa_decode_paged_workspace_size(pB, pHq, pHkv, table_np.shape[1], pps, pd, psplit)
     p_ws = torch.zeros(p_ws_bytes, dtype=torch.uint8, device=dev)  # arrival counters start at zero
+
+    def call_bwd():
+        fa.fa_bwd(q, k, v, o, b_do, lse, b_dq, b_dk, b_dv, B, Hq, Hkv, N, N, d, scale, 1, b_ws, b_ws_bytes, st)
 
     def call_paged():
         fa.fa_decode_paged(p_q, p_k, p_v, p_table, p_lens, p_o, p_lse, pB, pHq, pHkv, npages, pps,
@@ -311,6 +322,9 @@ def run_device(args):
     fwd_ms = timed_launches(call_fwd, args.steps, args.warmup) if do_fwd else [float("nan")]
     dec_ms = timed_launches(call_dec, args.steps, args.warmup) if do_dec else [float("nan")]
     paged_ms = timed_launches(call_paged, args.steps, args.warmup) if do_paged else [float("nan")]
+    if do_bwd and not do_fwd:
+        call_fwd()  # the backward consumes the forward's o and lse
+    bwd_ms = timed_launches(call_bwd, args.steps, args.warmup) if do_bwd else [float("nan")]
     if fa.fa_last_device_error(st) != fa.FA_OK:
         raise RuntimeError("device-side timeout recorded during the benchmark")
 
@@ -354,6 +368,7 @@ def run_device(args):
     fwd_mean = max_over_ranks(sum(fwd_ms) / len(fwd_ms), dev)
     dec_mean = max_over_ranks(sum(dec_ms) / len(dec_ms), dev)
     paged_mean = max_over_ranks(sum(paged_ms) / len(paged_ms), dev)
+    bwd_mean = max_over_ranks(sum(bwd_ms) / len(bwd_ms), dev)
     fwd_e2e_ms = max_over_ranks(fwd_e2e_ms, dev)
     dec_e2e_ms = max_over_ranks(dec_e2e_ms, dev)
     if world > 1:
@@ -374,6 +389,9 @@ def run_device(args):
     tc_peak = peaks["bf16"] if burst else peaks["bf16_sustained"]
     per_launch_tflops = F / (fwd_mean * 1e-3) / 1e12
     per_launch_gbs = kv / (dec_mean * 1e-3) / 1e9
+    bwd_flops = 2.5 * F
+    bwd_tflops = bwd_flops / (bwd_mean * 1e-3) / 1e12
+    bwd_peak = peaks["bf16"] if (args.steps * bwd_mean) < 1000.0 else peaks["bf16_sustained"]
     pkv = paged_kv_bytes(p_len)
     paged_gbs = pkv / (paged_mean * 1e-3) / 1e9
     cpu = cpu_baseline_fwd(args.cpu_seconds) if not args.no_cpu else None
@@ -422,12 +440,23 @@ def run_device(args):
                          "roofline": {"bound": "hbm", "achieved": round(paged_gbs, 1), "peak": peaks["hbm"],
                                       "unit": "GB/s", "frac": round(paged_gbs / peaks["hbm"], 4),
                                       "peak_kind": f"measured copy ({peaks['source']})",
+                                      "traffic": ncu_traffic("fa_decode_paged/decode_paged_ragged"),
                                       "kernels": "fa_decode_split_kernel<128,paged> (merge in-kernel)",
                                       "algorithmic_bytes_per_launch": pkv}},
+        "backward": {"value": round(aggregate_rate(bwd_flops, world, bwd_mean) / 1e12, 2), "unit": "TFLOP/s",
+                     "ms": round(bwd_mean, 4),
+                     "workload": "gqa_causal_8k backward (dQ, dK, dV from the forward's O and lse; dO seeded N(0,1))",
+                     "flops_convention": "2.5 x forward FLOPs (five products of the forward's two sizes)",
+                     "roofline": {"bound": "tensor", "achieved": round(bwd_tflops, 2), "peak": bwd_peak,
+                                  "unit": "TFLOP/s", "frac": round(bwd_tflops / bwd_peak, 4),
+                                  "peak_kind": f"measured ({peaks['source']})",
+                                  "traffic": ncu_traffic("fa_bwd/gqa_causal_8k"),
+                                  "kernels": "fa_bwd_pre_kernel<128> + fa_bwd_kernel<128> + fa_bwd_dq_kernel<128>",
+                                  "algorithmic_flops_per_launch": bwd_flops}},
         "e2e": {"value": round(world * F / (fwd_e2e_ms * 1e-3) / 1e12, 2), "unit": "TFLOP/s",
                 "h2d_bytes_per_step": h2d_fwd, "d2h_bytes_per_step": d2h_fwd},
         "cpu_baseline": cpu,
-        "gpu_launches": args.steps * (int(do_fwd) * 1 + int(do_dec) * 2 + int(do_paged) * 1)
+        "gpu_launches": args.steps * (int(do_fwd) * 1 + int(do_dec) * 2 + int(do_paged) * 1 + int(do_bwd) * 3)
         + (0 if args.no_e2e else e2e_steps * (int(do_fwd) * 1 + int(do_dec) * 2)),
         "clocks": clocks.summary(),
         "impl": "b200",
@@ -548,7 +577,7 @@ def main():
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--no-cpu", action="store_true", help="skip the CPU oracle baseline")
     ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer end-to-end phases")
-    ap.add_argument("--only", default="all", choices=["all", "fwd", "dec", "paged"],
+    ap.add_argument("--only", default="all", choices=["all", "fwd", "dec", "paged", "bwd"],
                     help="profiling: run one kernel family")
     args = ap.parse_args()
     if args.warmup < 3:
