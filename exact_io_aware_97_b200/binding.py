@@ -18,7 +18,7 @@ FA_OK, FA_ERR_INVALID_ARG, FA_ERR_UNSUPPORTED, FA_ERR_WORKSPACE, FA_ERR_CUDA, FA
 FA_BF16, FA_F32 = 0, 1
 
 EXPORTED = ("fa_fwd", "fa_fwd_workspace_size", "fa_decode", "fa_decode_workspace_size", "fa_decode_noalloc",
-            "fa_decode_paged", "fa_decode_paged_workspace_size", "fa_bwd", "fa_bwd_workspace_size",
+            "fa_decode_paged", "fa_decode_paged_workspace_size", "fa_bwd", "fa_bwd_workspace_size", "fa_fwd_qkvpacked",
             "fa_last_device_error", "fa_status_string", "fa_device_sm_count")
 FA_DECODE_NOALLOC_SCRATCH_BYTES = 16 << 20
 
@@ -55,6 +55,8 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
     L.fa_decode_paged.restype = i
     L.fa_decode_paged_workspace_size.argtypes = [i, i, i, i, i, i, i]
     L.fa_decode_paged_workspace_size.restype = sz
+    L.fa_fwd_qkvpacked.argtypes = [vp, vp, vp, i, i, i, i, f, i, vp, vp]
+    L.fa_fwd_qkvpacked.restype = i
     L.fa_bwd.argtypes = [vp] * 9 + [i] * 6 + [f, i, vp, sz, vp]
     L.fa_bwd.restype = i
     L.fa_bwd_workspace_size.argtypes = [i, i, i, i]
@@ -143,6 +145,12 @@ def fa_decode_paged(q, k_pages, v_pages, block_table, seqlens, o, lse, B, Hq, Hk
 def fa_decode_paged_workspace_size(B, Hq, Hkv, max_pages_per_seq, page_size, d, split_len) -> int:
     return int(load().fa_decode_paged_workspace_size(int(B), int(Hq), int(Hkv), int(max_pages_per_seq),
                                                      int(page_size), int(d), int(split_len)))
+
+
+def fa_fwd_qkvpacked(qkv, o, lse, B, H, N, d, scale, causal, cu_seqlens=None, stream=None) -> None:
+    st = load().fa_fwd_qkvpacked(_ptr(qkv), _ptr(o), _ptr(lse), int(B), int(H), int(N), int(d), float(scale),
+                                 int(bool(causal)), _ptr(cu_seqlens), _stream(stream))
+    _check(st, "fa_fwd_qkvpacked")
 
 
 def fa_bwd(q, k, v, o, dout, lse, dq, dk, dv, B, Hq, Hkv, Nq, Nk, d, scale, causal, workspace, workspace_bytes,
@@ -254,3 +262,21 @@ def backward(q, k, v, o, lse, dout, causal=False, scale=None, workspace=None, st
         workspace = torch.empty(max(ws_bytes, 1), dtype=torch.uint8, device=q.device)
     fa_bwd(q, k, v, o, dout, lse, dq, dk, dv, B, Hq, Hkv, Nq, Nk, d, scale, causal, workspace, ws_bytes, stream)
     return dq, dk, dv
+
+
+def forward_qkvpacked(qkv, causal=False, scale=None, cu_seqlens=None):
+    """O, lse for qkv [B,N,3,H,d] (or [total,3,H,d] with cu_seqlens), bf16."""
+    import torch
+    if cu_seqlens is not None:
+        total, _, H, d = qkv.shape
+        B, N = cu_seqlens.numel() - 1, total
+        out = torch.empty((total, H, d), dtype=torch.bfloat16, device=qkv.device)
+        lse = torch.empty((H, total), dtype=torch.float32, device=qkv.device)
+    else:
+        B, N, _, H, d = qkv.shape
+        out = torch.empty((B, N, H, d), dtype=torch.bfloat16, device=qkv.device)
+        lse = torch.empty((B, H, N), dtype=torch.float32, device=qkv.device)
+    if scale is None:
+        scale = d ** -0.5
+    fa_fwd_qkvpacked(qkv, out, lse, B, H, N, d, scale, causal, cu_seqlens)
+    return out, lse

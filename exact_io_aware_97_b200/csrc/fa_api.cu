@@ -49,12 +49,16 @@ EncodeTiledFn get_encode_fn() {
 }
 
 // [rows, heads, D] bf16 tensor (D innermost) seen as a 3-D map {D, heads, rows}; box of
-// 64 columns x 1 head x box_rows rows with the 128-byte swizzle.
-bool make_map(CUtensorMap* map, const void* base, int D, int heads, int64_t rows, int box_rows) {
+// 64 columns x 1 head x box_rows rows with the 128-byte swizzle.  Consecutive rows are
+// row_stride elements apart (heads * D when the tensor is dense; 3 * heads * D for one of
+// q, k, v inside a packed [rows, 3, heads, D] tensor).
+bool make_map(CUtensorMap* map, const void* base, int D, int heads, int64_t rows, int box_rows,
+              int64_t row_stride = 0) {
   EncodeTiledFn enc = get_encode_fn();
   if (!enc) return false;
+  if (row_stride <= 0) row_stride = (int64_t)heads * D;
   cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)heads, (cuuint64_t)rows};
-  cuuint64_t strides[2] = {(cuuint64_t)D * 2, (cuuint64_t)heads * D * 2};
+  cuuint64_t strides[2] = {(cuuint64_t)D * 2, (cuuint64_t)row_stride * 2};
   cuuint32_t box[3] = {64, 1, (cuuint32_t)box_rows};
   cuuint32_t estr[3] = {1, 1, 1};
   return enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
@@ -85,10 +89,10 @@ cudaError_t set_smem(K kernel, int bytes) {
 
 template <int D, bool F32>
 fa_status launch_fwd(const void* q, const void* k, const void* v, const FwdParams& prm, int64_t rows_q,
-                     int64_t rows_k, int units, cudaStream_t st) {
+                     int64_t rows_k, int units, cudaStream_t st, int64_t q_stride = 0, int64_t kv_stride = 0) {
   CUtensorMap mq, mk, mv;
-  if (!make_map(&mq, q, D, prm.Hq, rows_q, kBM) || !make_map(&mk, k, D, prm.Hkv, rows_k, kBN) ||
-      !make_map(&mv, v, D, prm.Hkv, rows_k, kBN))
+  if (!make_map(&mq, q, D, prm.Hq, rows_q, kBM, q_stride) || !make_map(&mk, k, D, prm.Hkv, rows_k, kBN, kv_stride) ||
+      !make_map(&mv, v, D, prm.Hkv, rows_k, kBN, kv_stride))
     return FA_ERR_CUDA;
   auto kern = fa_fwd_kernel<D, F32>;
   const int smem = FwdCfg<D>::kSmemBytes;
@@ -253,6 +257,44 @@ fa_status fa_fwd(const void* q, const void* k, const void* v, void* o, float* ls
                   : launch_fwd<64, false>(qb, kb, vb, prm, rows_q, rk, units, st);
   return f32out ? launch_fwd<128, true>(qb, kb, vb, prm, rows_q, rk, units, st)
                 : launch_fwd<128, false>(qb, kb, vb, prm, rows_q, rk, units, st);
+}
+
+fa_status fa_fwd_qkvpacked(const void* qkv, void* o, float* lse, int B, int H, int N, int d, float scale, int causal,
+                           const int32_t* cu_seqlens, void* stream) {
+  if (!qkv || !o) return FA_ERR_INVALID_ARG;
+  if (!aligned16(qkv) || !aligned16(o)) return FA_ERR_INVALID_ARG;
+  if (B < 0 || H <= 0 || N < 0) return FA_ERR_INVALID_ARG;
+  if (!(scale > 0.f) || !std::isfinite(scale)) return FA_ERR_INVALID_ARG;
+  if (d != 64 && d != 128) return FA_ERR_UNSUPPORTED;
+  const bool varlen = cu_seqlens != nullptr;
+  if (varlen) {
+    if (B > kMaxVarlenB || (int64_t)N > (int64_t)kMaxVarlenT * kUnitRows) return FA_ERR_UNSUPPORTED;
+    if ((reinterpret_cast<uintptr_t>(cu_seqlens) & 3u) != 0) return FA_ERR_INVALID_ARG;
+  }
+  const int64_t rows = varlen ? (int64_t)N : (int64_t)B * N;
+  if (rows >= (int64_t(1) << 31)) return FA_ERR_UNSUPPORTED;
+  if (B == 0 || N == 0) return FA_OK;
+  FwdParams prm{};
+  prm.o = o;
+  prm.lse = lse;
+  prm.cu = cu_seqlens;
+  prm.B = B;
+  prm.Hq = H;
+  prm.Hkv = H;
+  prm.G = 1;
+  prm.Nq = N;
+  prm.Nk = N;
+  prm.causal = causal ? 1 : 0;
+  prm.tau = (float)((double)scale * 1.4426950408889634074);
+  prm.T = varlen ? 0 : (N + kUnitRows - 1) / kUnitRows;
+  const int64_t units64 = varlen ? 0 : (int64_t)prm.T * B * H;
+  if (units64 >= (int64_t(1) << 31)) return FA_ERR_UNSUPPORTED;
+  const __nv_bfloat16* base = static_cast<const __nv_bfloat16*>(qkv);
+  const int64_t hd = (int64_t)H * d, stride = 3 * hd;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (d == 64)
+    return launch_fwd<64, false>(base, base + hd, base + 2 * hd, prm, rows, rows, (int)units64, st, stride, stride);
+  return launch_fwd<128, false>(base, base + hd, base + 2 * hd, prm, rows, rows, (int)units64, st, stride, stride);
 }
 
 size_t fa_decode_workspace_size(int B, int Hq, int Lmax, int d, int split_len) {

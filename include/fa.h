@@ -15,6 +15,7 @@
  *              section 4 "FlashDecoding"; "FlashAttention notes", section 4).
  *   fa_decode_paged  the same decode over a paged cache addressed through a block table.
  *   fa_bwd     the backward of fa_fwd by recomputation from the saved logsumexp.
+ *   fa_fwd_qkvpacked  fa_fwd reading q, k, v from one packed [.., 3, H, d] tensor.
  *
  * Conventions for every entry point:
  *   - All tensor pointers are DEVICE pointers owned by the caller.  The library never
@@ -83,6 +84,17 @@ FA_EXPORT fa_status fa_fwd(const void* q, const void* k, const void* v, void* o,
                  void* workspace, size_t workspace_bytes, void* stream);
 
 FA_EXPORT size_t fa_fwd_workspace_size(int B, int Hq, int Hkv, int Nq, int Nk, int d, fa_dtype in_dtype, int varlen);
+
+/* Forward attention on a packed qkv tensor (the flash_attn_qkvpacked_func interface of
+ * "Attention is All You Need부터 FlashAttention-3까지", section "practical implementation: using
+ * FlashAttention in PyTorch", whose example is qkv [2, 2048, 3, 12, 64], causal): q, k and v
+ * are the three slices of qkv [B, N, 3, H, d] bf16 (fixed length) or [total, 3, H, d] with
+ * cu_seqlens (variable length, as in fa_fwd, N = total rows).  H query heads and H key/value
+ * heads; o [B, N, H, d] (or [total, H, d]) bf16; lse as in fa_fwd (may be NULL).  Read in
+ * place through strided tensor maps: no copy, no workspace.  d 64 or 128; qkv and o 16-byte
+ * aligned. */
+FA_EXPORT fa_status fa_fwd_qkvpacked(const void* qkv, void* o, float* lse, int B, int H, int N, int d, float scale,
+                                     int causal, const int32_t* cu_seqlens, void* stream);
 
 /* Backward of fa_fwd (fixed length): gradients dq, dk, dv of o = attention(q, k, v) for an
  * upstream gradient dout of o ("FlashAttention notes", section 5.2 backward: P is rebuilt on
