@@ -19,6 +19,7 @@ FA_BF16, FA_F32 = 0, 1
 
 EXPORTED = ("fa_fwd", "fa_fwd_workspace_size", "fa_decode", "fa_decode_workspace_size", "fa_decode_noalloc",
             "fa_decode_paged", "fa_decode_paged_workspace_size", "fa_bwd", "fa_bwd_workspace_size", "fa_fwd_qkvpacked",
+            "fa_fwd_fp8", "fa_fwd_fp8_workspace_size",
             "fa_last_device_error", "fa_status_string", "fa_device_sm_count")
 FA_DECODE_NOALLOC_SCRATCH_BYTES = 16 << 20
 
@@ -55,6 +56,10 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
     L.fa_decode_paged.restype = i
     L.fa_decode_paged_workspace_size.argtypes = [i, i, i, i, i, i, i]
     L.fa_decode_paged_workspace_size.restype = sz
+    L.fa_fwd_fp8.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, i, f, f, f, f, i, vp, sz, vp]
+    L.fa_fwd_fp8.restype = i
+    L.fa_fwd_fp8_workspace_size.argtypes = [i, i, i, i]
+    L.fa_fwd_fp8_workspace_size.restype = sz
     L.fa_fwd_qkvpacked.argtypes = [vp, vp, vp, i, i, i, i, f, i, vp, vp]
     L.fa_fwd_qkvpacked.restype = i
     L.fa_bwd.argtypes = [vp] * 9 + [i] * 6 + [f, i, vp, sz, vp]
@@ -145,6 +150,18 @@ def fa_decode_paged(q, k_pages, v_pages, block_table, seqlens, o, lse, B, Hq, Hk
 def fa_decode_paged_workspace_size(B, Hq, Hkv, max_pages_per_seq, page_size, d, split_len) -> int:
     return int(load().fa_decode_paged_workspace_size(int(B), int(Hq), int(Hkv), int(max_pages_per_seq),
                                                      int(page_size), int(d), int(split_len)))
+
+
+def fa_fwd_fp8(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, d, scale, descale_q, descale_k, descale_v, causal, workspace,
+               workspace_bytes, stream=None) -> None:
+    st = load().fa_fwd_fp8(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), int(B), int(Hq), int(Hkv), int(Nq),
+                           int(Nk), int(d), float(scale), float(descale_q), float(descale_k), float(descale_v),
+                           int(bool(causal)), _ptr(workspace), int(workspace_bytes), _stream(stream))
+    _check(st, "fa_fwd_fp8")
+
+
+def fa_fwd_fp8_workspace_size(B, Hkv, Nk, d) -> int:
+    return int(load().fa_fwd_fp8_workspace_size(int(B), int(Hkv), int(Nk), int(d)))
 
 
 def fa_fwd_qkvpacked(qkv, o, lse, B, H, N, d, scale, causal, cu_seqlens=None, stream=None) -> None:
@@ -280,3 +297,20 @@ def forward_qkvpacked(qkv, causal=False, scale=None, cu_seqlens=None):
         scale = d ** -0.5
     fa_fwd_qkvpacked(qkv, out, lse, B, H, N, d, scale, causal, cu_seqlens)
     return out, lse
+
+
+def forward_fp8(q8, k8, v8, descale_q, descale_k, descale_v, causal=False, scale=None, workspace=None):
+    """O (bf16), lse for e4m3 q8 [B,Nq,Hq,128], k8/v8 [B,Nk,Hkv,128] (uint8 or float8 tensors)."""
+    import torch
+    B, Nq, Hq, d = q8.shape
+    Nk, Hkv = k8.shape[1], k8.shape[2]
+    if scale is None:
+        scale = d ** -0.5
+    o = torch.empty((B, Nq, Hq, d), dtype=torch.bfloat16, device=q8.device)
+    lse = torch.empty((B, Hq, Nq), dtype=torch.float32, device=q8.device)
+    ws_bytes = fa_fwd_fp8_workspace_size(B, Hkv, Nk, d)
+    if workspace is None:
+        workspace = torch.empty(max(ws_bytes, 1), dtype=torch.uint8, device=q8.device)
+    fa_fwd_fp8(q8, k8, v8, o, lse, B, Hq, Hkv, Nq, Nk, d, scale, descale_q, descale_k, descale_v, causal, workspace,
+               ws_bytes)
+    return o, lse

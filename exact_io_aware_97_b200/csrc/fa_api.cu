@@ -29,6 +29,31 @@ __global__ void cast_f32_bf16_kernel(const float* __restrict__ src, __nv_bfloat1
     dst[i] = __float2bfloat16_rn(src[i]);
 }
 
+// V^T for the fp8 forward: vt[(b*Hkv + h)*128 + c][n] = v[b][n][h][c] for n < Nk, 0 up to
+// NkPad (so that padded keys hold finite values; they are masked).  One block per (64-key
+// chunk, head, sequence), staged through shared memory so both sides are coalesced.
+__global__ void __launch_bounds__(256) transpose_v_e4m3_kernel(const uint8_t* __restrict__ v, uint8_t* __restrict__ vt,
+                                                               int Nk, int Hkv, int NkPad) {
+  __shared__ uint32_t tile[64][33];  // 64 keys x 128 bytes (32 words), padded
+  const int n0 = blockIdx.x * 64, h = blockIdx.y, b = blockIdx.z;
+  for (int idx = threadIdx.x; idx < 64 * 32; idx += 256) {
+    const int r = idx >> 5, w = idx & 31;
+    const int n = n0 + r;
+    tile[r][w] = (n < Nk) ? reinterpret_cast<const uint32_t*>(v + (((size_t)b * Nk + n) * Hkv + h) * 128)[w] : 0u;
+  }
+  __syncthreads();
+  // each thread writes 4 consecutive keys (one word) of one column c
+  for (int idx = threadIdx.x; idx < 128 * 16; idx += 256) {
+    const int c = idx >> 4, kq = idx & 15;  // column, group of four keys
+    const int n = n0 + 4 * kq;
+    if (n >= NkPad) continue;
+    uint32_t word = 0;
+#pragma unroll
+    for (int e = 0; e < 4; ++e) word |= ((tile[4 * kq + e][c >> 2] >> (8 * (c & 3))) & 0xFFu) << (8 * e);
+    *reinterpret_cast<uint32_t*>(vt + (((size_t)b * Hkv + h) * 128 + c) * NkPad + n) = word;
+  }
+}
+
 namespace {
 
 using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
@@ -62,6 +87,17 @@ bool make_map(CUtensorMap* map, const void* base, int D, int heads, int64_t rows
   cuuint32_t box[3] = {64, 1, (cuuint32_t)box_rows};
   cuuint32_t estr[3] = {1, 1, 1};
   return enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// Byte tensor (e4m3 stored as bytes) of three dimensions with the 128-byte swizzle.
+bool make_map_u8(CUtensorMap* map, const void* base, const cuuint64_t (&dims)[3], const cuuint64_t (&strides)[2],
+                 const cuuint32_t (&box)[3]) {
+  EncodeTiledFn enc = get_encode_fn();
+  if (!enc) return false;
+  cuuint32_t estr[3] = {1, 1, 1};
+  return enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void*>(base), dims, strides, box, estr,
              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
@@ -245,6 +281,7 @@ fa_status fa_fwd(const void* q, const void* k, const void* v, void* o, float* ls
   prm.Nk = Nk;
   prm.causal = causal ? 1 : 0;
   prm.tau = (float)((double)scale * 1.4426950408889634074);
+  prm.o_scale = 1.f;
   prm.T = varlen ? 0 : (Nq + kUnitRows - 1) / kUnitRows;
   const int64_t units64 = varlen ? 0 : (int64_t)prm.T * B * Hq;
   if (units64 >= (int64_t(1) << 31)) return FA_ERR_UNSUPPORTED;
@@ -257,6 +294,74 @@ fa_status fa_fwd(const void* q, const void* k, const void* v, void* o, float* ls
                   : launch_fwd<64, false>(qb, kb, vb, prm, rows_q, rk, units, st);
   return f32out ? launch_fwd<128, true>(qb, kb, vb, prm, rows_q, rk, units, st)
                 : launch_fwd<128, false>(qb, kb, vb, prm, rows_q, rk, units, st);
+}
+
+size_t fa_fwd_fp8_workspace_size(int B, int Hkv, int Nk, int d) {
+  if (B <= 0 || Hkv <= 0 || Nk <= 0 || d != 128) return 0;
+  const size_t pad = (size_t)(Nk + 15) / 16 * 16;
+  return align_up((size_t)B * Hkv * d * pad, 256);
+}
+
+fa_status fa_fwd_fp8(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq, int Hkv,
+                     int Nq, int Nk, int d, float scale, float descale_q, float descale_k, float descale_v,
+                     int causal, void* workspace, size_t workspace_bytes, void* stream) {
+  if (!q || !k || !v || !o) return FA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o)) return FA_ERR_INVALID_ARG;
+  if (B < 0 || Hq <= 0 || Hkv <= 0 || Nq < 0 || Nk < 0) return FA_ERR_INVALID_ARG;
+  for (float x : {scale, descale_q, descale_k, descale_v})
+    if (!(x > 0.f) || !std::isfinite(x)) return FA_ERR_INVALID_ARG;
+  if (Hq % Hkv != 0) return FA_ERR_UNSUPPORTED;
+  if (d != 128) return FA_ERR_UNSUPPORTED;
+  const int64_t rows_q = (int64_t)B * Nq, rows_k = (int64_t)B * Nk;
+  if (rows_q >= (int64_t(1) << 31) || rows_k >= (int64_t(1) << 31)) return FA_ERR_UNSUPPORTED;
+  if (B > 65535 || Hkv > 65535) return FA_ERR_UNSUPPORTED;
+  if (B == 0 || Nq == 0) return FA_OK;
+  const int pad = (Nk + 15) / 16 * 16;
+  const size_t need = fa_fwd_fp8_workspace_size(B, Hkv, Nk, d);
+  if (need > 0 && (!workspace || workspace_bytes < need || !aligned16(workspace))) return FA_ERR_WORKSPACE;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  uint8_t* vt = static_cast<uint8_t*>(workspace);
+  if (Nk > 0) {
+    dim3 g((pad + 63) / 64, Hkv, B);
+    transpose_v_e4m3_kernel<<<g, 256, 0, st>>>(static_cast<const uint8_t*>(v), vt, Nk, Hkv, pad);
+    if (cudaGetLastError() != cudaSuccess) return FA_ERR_CUDA;
+  }
+  FwdParams prm{};
+  prm.o = o;
+  prm.lse = lse;
+  prm.cu = nullptr;
+  prm.B = B;
+  prm.Hq = Hq;
+  prm.Hkv = Hkv;
+  prm.G = Hq / Hkv;
+  prm.Nq = Nq;
+  prm.Nk = Nk;
+  prm.causal = causal ? 1 : 0;
+  prm.tau = (float)((double)scale * descale_q * descale_k * 1.4426950408889634074);
+  prm.o_scale = descale_v;
+  prm.T = (Nq + kUnitRows - 1) / kUnitRows;
+  const int64_t units64 = (int64_t)prm.T * B * Hq;
+  if (units64 >= (int64_t(1) << 31)) return FA_ERR_UNSUPPORTED;
+  CUtensorMap mq, mk, mv;
+  const cuuint64_t dq3[3] = {128, (cuuint64_t)Hq, (cuuint64_t)rows_q};
+  const cuuint64_t sq2[2] = {128, (cuuint64_t)Hq * 128};
+  const cuuint64_t dk3[3] = {128, (cuuint64_t)Hkv, (cuuint64_t)std::max<int64_t>(rows_k, 1)};
+  const cuuint64_t sk2[2] = {128, (cuuint64_t)Hkv * 128};
+  const cuuint64_t dv3[3] = {(cuuint64_t)std::max(pad, 16), 128, (cuuint64_t)B * Hkv};
+  const cuuint64_t sv2[2] = {(cuuint64_t)std::max(pad, 16), (cuuint64_t)std::max(pad, 16) * 128};
+  const cuuint32_t box_rows[3] = {128, 1, (cuuint32_t)kBM};
+  const cuuint32_t box_vt[3] = {(cuuint32_t)kBN, 128, 1};
+  if (!make_map_u8(&mq, q, dq3, sq2, box_rows) || !make_map_u8(&mk, k, dk3, sk2, box_rows) ||
+      !make_map_u8(&mv, Nk > 0 ? (const void*)vt : k, dv3, sv2, box_vt))
+    return FA_ERR_CUDA;
+  auto kern = fa_fwd_kernel<128, false, true>;
+  const int smem = FwdCfg<128, true>::kSmemBytes;
+  if (set_smem(kern, smem) != cudaSuccess) return FA_ERR_CUDA;
+  const int sms = sm_count_cached();
+  if (sms <= 0) return FA_ERR_CUDA;
+  const int units = (int)units64;
+  kern<<<std::min(units, sms), kFwdThreads, smem, st>>>(mq, mk, mv, prm);
+  return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
 
 fa_status fa_fwd_qkvpacked(const void* qkv, void* o, float* lse, int B, int H, int N, int d, float scale, int causal,
@@ -286,6 +391,7 @@ fa_status fa_fwd_qkvpacked(const void* qkv, void* o, float* lse, int B, int H, i
   prm.Nk = N;
   prm.causal = causal ? 1 : 0;
   prm.tau = (float)((double)scale * 1.4426950408889634074);
+  prm.o_scale = 1.f;
   prm.T = varlen ? 0 : (N + kUnitRows - 1) / kUnitRows;
   const int64_t units64 = varlen ? 0 : (int64_t)prm.T * B * H;
   if (units64 >= (int64_t(1) << 31)) return FA_ERR_UNSUPPORTED;

@@ -39,8 +39,9 @@ struct FwdParams {
   const int32_t* cu;  // varlen offsets [B+1] or null
   int B, Hq, Hkv, G, Nq, Nk;
   int causal;
-  float tau;  // scale * log2(e)
-  int T;      // fixed length: 256-row units per (sequence, head)
+  float tau;      // scale * log2(e) (fp8: times the q and k dequantisation factors)
+  float o_scale;  // multiplies O at the end (fp8: the v dequantisation factor; else 1)
+  int T;          // fixed length: 256-row units per (sequence, head)
 };
 
 constexpr int kBM = 128;        // query rows per tile
@@ -62,11 +63,16 @@ constexpr float kRescaleThreshold = 8.0f;
 constexpr uint32_t kEmuPairMask = 0x00;
 constexpr uint32_t kIntPackPairMask = 0x00;
 
-template <int D>
+// FP8: q, k, v in e4m3 (d = 128 only), the S and P V products on the kind::f8f6f4 tensor-core
+// path with P rounded to e4m3, V read from a [d, keys] transposed copy so that both operands
+// of P V are K-major.
+template <int D, bool FP8 = false>
 struct FwdCfg {
-  static constexpr int kTileBytes = kBM * D * 2;  // one 128 x D bf16 tile
-  static constexpr int kChunkBytes = kBM * 128;   // one 128-row x 64-column swizzle panel
-  static constexpr int kStages = (D == 128) ? 4 : 8;
+  static constexpr int kTileBytes = kBM * D * (FP8 ? 1 : 2);  // one 128 x D tile
+  static constexpr int kChunkBytes = kBM * 128;                // one 128-row x 128-byte swizzle panel
+  static constexpr int kPanels = kTileBytes / kChunkBytes;
+  static constexpr int kPanelCols = FP8 ? 128 : 64;            // elements per 128-byte panel row
+  static constexpr int kStages = (FP8 || D == 64) ? 8 : 4;
   static constexpr int kQBytes = 2 * kTileBytes;
   static constexpr int kRingBytes = kStages * kTileBytes;
   static constexpr int kNumBars = 2 + 2 * kStages + 10;
@@ -166,11 +172,12 @@ struct UnitIter {
   }
 };
 
-template <int D, bool OUT_F32>
+template <int D, bool OUT_F32, bool FP8 = false>
 __global__ void __launch_bounds__(kFwdThreads, 1)
     fa_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                   const __grid_constant__ CUtensorMap tmV, const FwdParams p) {
-  using C = FwdCfg<D>;
+  static_assert(!FP8 || (D == 128 && !OUT_F32), "fp8 forward: d = 128, bf16 output");
+  using C = FwdCfg<D, FP8>;
   constexpr int NS = C::kStages;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -287,8 +294,8 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         const int ntile = un.valid[1] ? 2 : 1;
         mbar_arrive_expect_tx_elect(q_full, ntile * C::kTileBytes);
         for (int i = 0; i < ntile; ++i)
-          for (int c = 0; c < D / 64; ++c)
-            tma_load_3d_elect(sQ + i * C::kTileBytes + c * C::kChunkBytes, &tmQ, c * 64, un.h,
+          for (int c = 0; c < C::kPanels; ++c)
+            tma_load_3d_elect(sQ + i * C::kTileBytes + c * C::kChunkBytes, &tmQ, c * C::kPanelCols, un.h,
                         un.q_start + un.row0 + i * kBM, q_full);
         for (int j = 0; j < un.nmax && ok; ++j) {
           for (int kv = 0; kv < 2; ++kv) {
@@ -298,9 +305,15 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
               break;
             }
             mbar_arrive_expect_tx_elect(full + slot, C::kTileBytes);
-            for (int c = 0; c < D / 64; ++c)
-              tma_load_3d_hint_elect(sRing + slot * C::kTileBytes + c * C::kChunkBytes, kv ? &tmV : &tmK, c * 64,
-                               un.kvh, un.k_start + j * kBN, full + slot, kv_policy);
+            if (FP8 && kv) {
+              // V^T tile: d rows of 128 keys from the [B * Hkv, d, keys] transposed copy
+              tma_load_3d_hint_elect(sRing + slot * C::kTileBytes, &tmV, j * kBN, 0, un.b * p.Hkv + un.kvh,
+                                     full + slot, kv_policy);
+            } else {
+              for (int c = 0; c < C::kPanels; ++c)
+                tma_load_3d_hint_elect(sRing + slot * C::kTileBytes + c * C::kChunkBytes, kv ? &tmV : &tmK,
+                                       c * C::kPanelCols, un.kvh, un.k_start + j * kBN, full + slot, kv_policy);
+            }
             ++g;
           }
         }
@@ -311,8 +324,8 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
   } else if (warp == 8) {
     // ================================================================ MMA issuer
     {
-      constexpr uint32_t idS = idesc_bf16_f32(kBM, kBN, false);
-      constexpr uint32_t idPV = idesc_bf16_f32(kBM, D, true);
+      constexpr uint32_t idS = FP8 ? idesc_e4m3_f32(kBM, kBN) : idesc_bf16_f32(kBM, kBN, false);
+      constexpr uint32_t idPV = FP8 ? idesc_e4m3_f32(kBM, D) : idesc_bf16_f32(kBM, D, true);
       const uint32_t qbase = smem_u32(sQ);
       const uint32_t rbase = smem_u32(sRing);
       uint32_t g = 0, qcount = 0;
@@ -321,22 +334,36 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       UnitWalker wk;
       bool ok = true;
 
+      // k-steps of 32 bytes along d (16 bf16 or 32 e4m3 elements), four per 128-byte panel
       auto issue_S = [&](int i, uint32_t slot) {
 #pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
+        for (int kk = 0; kk < D * (FP8 ? 1 : 2) / 32; ++kk) {
           const uint32_t off = (kk >> 2) * C::kChunkBytes + (kk & 3) * 32;
           const uint64_t a = smem_desc_sw128(qbase + i * C::kTileBytes + off, 16, 1024);
           const uint64_t bd = smem_desc_sw128(rbase + slot * C::kTileBytes + off, 16, 1024);
-          umma_ss_elect(tmem + i * kBN, a, bd, idS, kk > 0 ? 1u : 0u);
+          if (FP8)
+            umma_ss_f8_elect(tmem + i * kBN, a, bd, idS, kk > 0 ? 1u : 0u);
+          else
+            umma_ss_elect(tmem + i * kBN, a, bd, idS, kk > 0 ? 1u : 0u);
         }
       };
       // O_i (+)= P_i V for the keys of one half (8 k-steps of 16 keys in all).
+      // (P in TMEM: 8 columns per k-step either way, 16 keys of bf16 or 32 keys of e4m3)
       auto issue_PV_half = [&](int i, uint32_t slot, int half, bool acc) {
+        if (FP8) {
 #pragma unroll
-        for (int k4 = 0; k4 < kBN / 32; ++k4) {
-          const int kk = half * (kBN / 32) + k4;
-          const uint64_t bd = smem_desc_sw128(rbase + slot * C::kTileBytes + kk * 16 * 128, C::kChunkBytes, 1024);
-          umma_ts_elect(tmem + C::kColO + i * D, tmem + i * kBN + kk * 8, bd, idPV, (acc || kk > 0) ? 1u : 0u);
+          for (int k2 = 0; k2 < kBN / 64; ++k2) {
+            const int kk = half * (kBN / 64) + k2;  // 32 keys = 32 bytes of each V^T row
+            const uint64_t bd = smem_desc_sw128(rbase + slot * C::kTileBytes + kk * 32, 16, 1024);
+            umma_ts_f8_elect(tmem + C::kColO + i * D, tmem + i * kBN + kk * 8, bd, idPV, (acc || kk > 0) ? 1u : 0u);
+          }
+        } else {
+#pragma unroll
+          for (int k4 = 0; k4 < kBN / 32; ++k4) {
+            const int kk = half * (kBN / 32) + k4;
+            const uint64_t bd = smem_desc_sw128(rbase + slot * C::kTileBytes + kk * 16 * 128, C::kChunkBytes, 1024);
+            umma_ts_elect(tmem + C::kColO + i * D, tmem + i * kBN + kk * 8, bd, idPV, (acc || kk > 0) ? 1u : 0u);
+          }
         }
       };
       auto wait_full = [&](uint32_t gi) -> bool {
@@ -497,22 +524,39 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         uint64_t lsum[2] = {f2(0.f, 0.f), f2(0.f, 0.f)};
 #pragma unroll
         for (int half = 0; half < 2; ++half) {
-          uint32_t pk[32];
+          if (FP8) {
+            // e4m3 P, four keys per TMEM column: 64 keys in 16 columns
+            uint32_t pk[16];
 #pragma unroll
-          for (int e = 0; e < 32; ++e) {
-            const int g = 32 * half + e;  // column pair
-            float x0, x1, p0, p1;
-            f2_split(f2_fma(f2(s[2 * g], s[2 * g + 1]), tau2, nms2), x0, x1);
-            if (((kEmuPairMask >> (g & 7)) & 1u) && !need_mask) {
-              exp2_poly_x2(x0, x1, p0, p1);
-            } else {
-              p0 = ex2_approx(x0);
-              p1 = ex2_approx(x1);
+            for (int e = 0; e < 16; ++e) {
+              const int g = 32 * half + 2 * e;  // first of two column pairs
+              float x0, x1, x2, x3;
+              f2_split(f2_fma(f2(s[2 * g], s[2 * g + 1]), tau2, nms2), x0, x1);
+              f2_split(f2_fma(f2(s[2 * g + 2], s[2 * g + 3]), tau2, nms2), x2, x3);
+              const float p0 = ex2_approx(x0), p1 = ex2_approx(x1), p2 = ex2_approx(x2), p3 = ex2_approx(x3);
+              lsum[0] = f2_add(lsum[0], f2(p0, p1));
+              lsum[1] = f2_add(lsum[1], f2(p2, p3));
+              pk[e] = pack_e4m3x4(p0, p1, p2, p3);
             }
-            lsum[g & 1] = f2_add(lsum[g & 1], f2(p0, p1));
-            pk[e] = ((kIntPackPairMask >> (g & 7)) & 1u) ? pack_bf16x2_int(p0, p1) : pack_bf16x2(p0, p1);
+            tmem_st16(tS + 16 * half, pk);
+          } else {
+            uint32_t pk[32];
+#pragma unroll
+            for (int e = 0; e < 32; ++e) {
+              const int g = 32 * half + e;  // column pair
+              float x0, x1, p0, p1;
+              f2_split(f2_fma(f2(s[2 * g], s[2 * g + 1]), tau2, nms2), x0, x1);
+              if (((kEmuPairMask >> (g & 7)) & 1u) && !need_mask) {
+                exp2_poly_x2(x0, x1, p0, p1);
+              } else {
+                p0 = ex2_approx(x0);
+                p1 = ex2_approx(x1);
+              }
+              lsum[g & 1] = f2_add(lsum[g & 1], f2(p0, p1));
+              pk[e] = ((kIntPackPairMask >> (g & 7)) & 1u) ? pack_bf16x2_int(p0, p1) : pack_bf16x2(p0, p1);
+            }
+            tmem_st32(tS + 32 * half, pk);
           }
-          tmem_st32(tS + 32 * half, pk);
           tmem_wait_st();
           tc_fence_before();
           mbar_arrive(p_half + 2 * i + half);
@@ -531,7 +575,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       }
       pvcnt += n;
       const bool row_ok = row < un.nq;
-      const float inv_l = l > 0.f ? 1.f / l : 0.f;
+      const float inv_l = l > 0.f ? p.o_scale / l : 0.f;
       const size_t orow = ((size_t)(un.q_start + row) * p.Hq + un.h) * D;
 #pragma unroll
       for (int c = 0; c < D / 32; ++c) {

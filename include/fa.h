@@ -16,6 +16,7 @@
  *   fa_decode_paged  the same decode over a paged cache addressed through a block table.
  *   fa_bwd     the backward of fa_fwd by recomputation from the saved logsumexp.
  *   fa_fwd_qkvpacked  fa_fwd reading q, k, v from one packed [.., 3, H, d] tensor.
+ *   fa_fwd_fp8 the forward on e4m3 inputs with per-tensor scales.
  *
  * Conventions for every entry point:
  *   - All tensor pointers are DEVICE pointers owned by the caller.  The library never
@@ -84,6 +85,25 @@ FA_EXPORT fa_status fa_fwd(const void* q, const void* k, const void* v, void* o,
                  void* workspace, size_t workspace_bytes, void* stream);
 
 FA_EXPORT size_t fa_fwd_workspace_size(int B, int Hq, int Hkv, int Nq, int Nk, int d, fa_dtype in_dtype, int varlen);
+
+/* FP8 forward ("Attention is All You Need부터 FlashAttention-3까지", FlashAttention-3 section:
+ * FP8 support for higher throughput; "FlashAttention-3 (FA-3)", section 2 feature table: FP8):
+ * q, k, v are e4m3 (OCP FP8, stored one byte each) with per-tensor dequantisation factors:
+ * the value of an element is (its e4m3 value) * descale_x.  Computes the same O and lse as
+ * fa_fwd for the dequantised inputs: S = q k^T on the e4m3 tensor-core path (fp32
+ * accumulation, exact products), softmax in fp32, P rounded to e4m3 (nearest even, values
+ * <= 256 by the lazy rescale) for the P V product, l summed from the unrounded P; O is written
+ * as bf16, lse as in fa_fwd.  Fixed length; d must be 128.
+ * q [B, Nq, Hq, 128], k and v [B, Nk, Hkv, 128] (bytes), o [B, Nq, Hq, 128] bf16,
+ * lse [B, Hq, Nq] fp32 (may be NULL).  Same causal rule and head grouping as fa_fwd.
+ * workspace: at least fa_fwd_fp8_workspace_size(B, Hkv, Nk, 128) bytes; it receives a
+ * transposed copy of v ([B, Hkv, 128, Nk rounded up to 16]) so that both operands of P V are
+ * K-major. */
+FA_EXPORT fa_status fa_fwd_fp8(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq,
+                               int Hkv, int Nq, int Nk, int d, float scale, float descale_q, float descale_k,
+                               float descale_v, int causal, void* workspace, size_t workspace_bytes, void* stream);
+
+FA_EXPORT size_t fa_fwd_fp8_workspace_size(int B, int Hkv, int Nk, int d);
 
 /* Forward attention on a packed qkv tensor (the flash_attn_qkvpacked_func interface of
  * "Attention is All You Need부터 FlashAttention-3까지", section "practical implementation: using

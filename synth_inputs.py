@@ -123,6 +123,19 @@ def cu_seqlens(lengths) -> np.ndarray:
     return cu
 
 
+def to_e4m3(x: np.ndarray):
+    """Per-tensor e4m3 storage of float32 values: the scale maps the largest magnitude to 448
+    (the largest finite e4m3 value); returns (bytes uint8, dequantised float32 values, scale),
+    with value = e4m3(byte) * scale.  Conversion: torch's float8_e4m3fn cast (round to nearest
+    even, saturating)."""
+    import torch
+    x = np.ascontiguousarray(x, dtype=np.float32)
+    amax = float(np.abs(x).max()) if x.size else 0.0
+    scale = amax / 448.0 if amax > 0 else 1.0
+    f8 = torch.from_numpy(x / np.float32(scale)).to(torch.float8_e4m3fn)
+    return f8.view(torch.uint8).numpy().copy(), (f8.to(torch.float32).numpy() * np.float32(scale)), scale
+
+
 def permutation(seed: int, tensor_id: int, n: int) -> np.ndarray:
     """A permutation of 0..n-1: the indices that sort n words of the stream (stable)."""
     return np.argsort(words(stream_key(seed, tensor_id), 0, n), kind="stable").astype(np.int64)
