@@ -242,6 +242,7 @@ def run_device(args):
     do_dec = args.only in ("all", "dec")
     do_paged = args.only in ("all", "paged")
     do_bwd = args.only in ("all", "bwd")
+    do_fp8 = args.only in ("all", "fp8")
     if do_bwd:
         h_do_f = torch.from_numpy(inputs("fwd", seed, DOUT_ID, (B, N, Hq, d))).to(torch.bfloat16)
         b_do = h_do_f.to(dev)
@@ -284,6 +285,20 @@ def run_device(args):
     p_ws_bytes = fa.fa_decode_paged_workspace_size(pB, pHq, pHkv, table_np.shape[1], pps, pd, psplit)
     p_ws = torch.zeros(p_ws_bytes, dtype=torch.uint8, device=dev)  # arrival counters start at zero
 
+    if do_fp8:
+        f8 = [si.to_e4m3(inputs("fwd", seed, tid, shp)) for tid, shp in
+              ((si.Q, (B, N, Hq, d)), (si.K, (B, N, Hkv, d)), (si.V, (B, N, Hkv, d)))]
+        f8_q, f8_k, f8_v = (torch.from_numpy(t[0]).to(dev) for t in f8)
+        f8_desc = [t[2] for t in f8]
+        f8_o = torch.empty((B, N, Hq, d), dtype=torch.bfloat16, device=dev)
+        f8_lse = torch.empty((B, Hq, N), dtype=torch.float32, device=dev)
+        f8_ws_bytes = fa.fa_fwd_fp8_workspace_size(B, Hkv, N, d)
+        f8_ws = torch.empty(f8_ws_bytes, dtype=torch.uint8, device=dev)
+
+    def call_fp8():
+        fa.fa_fwd_fp8(f8_q, f8_k, f8_v, f8_o, f8_lse, B, Hq, Hkv, N, N, d, scale, f8_desc[0], f8_desc[1], f8_desc[2],
+                      1, f8_ws, f8_ws_bytes, st)
+
     def call_bwd():
         fa.fa_bwd(q, k, v, o, b_do, lse, b_dq, b_dk, b_dv, B, Hq, Hkv, N, N, d, scale, 1, b_ws, b_ws_bytes, st)
 
@@ -325,6 +340,7 @@ def run_device(args):
     if do_bwd and not do_fwd:
         call_fwd()  # the backward consumes the forward's o and lse
     bwd_ms = timed_launches(call_bwd, args.steps, args.warmup) if do_bwd else [float("nan")]
+    fp8_ms = timed_launches(call_fp8, args.steps, args.warmup) if do_fp8 else [float("nan")]
     if fa.fa_last_device_error(st) != fa.FA_OK:
         raise RuntimeError("device-side timeout recorded during the benchmark")
 
@@ -369,6 +385,7 @@ def run_device(args):
     dec_mean = max_over_ranks(sum(dec_ms) / len(dec_ms), dev)
     paged_mean = max_over_ranks(sum(paged_ms) / len(paged_ms), dev)
     bwd_mean = max_over_ranks(sum(bwd_ms) / len(bwd_ms), dev)
+    fp8_mean = max_over_ranks(sum(fp8_ms) / len(fp8_ms), dev)
     fwd_e2e_ms = max_over_ranks(fwd_e2e_ms, dev)
     dec_e2e_ms = max_over_ranks(dec_e2e_ms, dev)
     if world > 1:
@@ -392,6 +409,8 @@ def run_device(args):
     bwd_flops = 2.5 * F
     bwd_tflops = bwd_flops / (bwd_mean * 1e-3) / 1e12
     bwd_peak = peaks["bf16"] if (args.steps * bwd_mean) < 1000.0 else peaks["bf16_sustained"]
+    fp8_tflops = F / (fp8_mean * 1e-3) / 1e12
+    fp8_peak = 2.0 * (peaks["bf16"] if (args.steps * fp8_mean) < 1000.0 else peaks["bf16_sustained"])
     pkv = paged_kv_bytes(p_len)
     paged_gbs = pkv / (paged_mean * 1e-3) / 1e9
     cpu = cpu_baseline_fwd(args.cpu_seconds) if not args.no_cpu else None
@@ -443,6 +462,15 @@ def run_device(args):
                                       "traffic": ncu_traffic("fa_decode_paged/decode_paged_ragged"),
                                       "kernels": "fa_decode_split_kernel<128,paged> (merge in-kernel)",
                                       "algorithmic_bytes_per_launch": pkv}},
+        "forward_fp8": {"value": round(aggregate_rate(F, world, fp8_mean) / 1e12, 2), "unit": "TFLOP/s",
+                        "ms": round(fp8_mean, 4),
+                        "workload": "gqa_causal_8k with e4m3 q, k, v (per-tensor scales), P in e4m3, O bf16",
+                        "roofline": {"bound": "tensor", "achieved": round(fp8_tflops, 2), "peak": round(fp8_peak, 1),
+                                     "unit": "TFLOP/s", "frac": round(fp8_tflops / fp8_peak, 4),
+                                     "peak_kind": f"measured bf16 x 2 (nominal fp8/bf16 ratio; {peaks['source']})",
+                                     "traffic": ncu_traffic("fa_fwd_fp8/gqa_causal_8k"),
+                                     "kernels": "transpose_v_e4m3_kernel + fa_fwd_kernel<128,false,fp8>",
+                                     "algorithmic_flops_per_launch": F}},
         "backward": {"value": round(aggregate_rate(bwd_flops, world, bwd_mean) / 1e12, 2), "unit": "TFLOP/s",
                      "ms": round(bwd_mean, 4),
                      "workload": "gqa_causal_8k backward (dQ, dK, dV from the forward's O and lse; dO seeded N(0,1))",
@@ -456,7 +484,7 @@ def run_device(args):
         "e2e": {"value": round(world * F / (fwd_e2e_ms * 1e-3) / 1e12, 2), "unit": "TFLOP/s",
                 "h2d_bytes_per_step": h2d_fwd, "d2h_bytes_per_step": d2h_fwd},
         "cpu_baseline": cpu,
-        "gpu_launches": args.steps * (int(do_fwd) * 1 + int(do_dec) * 2 + int(do_paged) * 1 + int(do_bwd) * 3)
+        "gpu_launches": args.steps * (int(do_fwd) * 1 + int(do_dec) * 2 + int(do_paged) * 1 + int(do_bwd) * 3 + int(do_fp8) * 2)
         + (0 if args.no_e2e else e2e_steps * (int(do_fwd) * 1 + int(do_dec) * 2)),
         "clocks": clocks.summary(),
         "impl": "b200",
@@ -577,7 +605,7 @@ def main():
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--no-cpu", action="store_true", help="skip the CPU oracle baseline")
     ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer end-to-end phases")
-    ap.add_argument("--only", default="all", choices=["all", "fwd", "dec", "paged", "bwd"],
+    ap.add_argument("--only", default="all", choices=["all", "fwd", "dec", "paged", "bwd", "fp8"],
                     help="profiling: run one kernel family")
     args = ap.parse_args()
     if args.warmup < 3:
