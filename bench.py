@@ -489,7 +489,18 @@ def run_device(args):
         "clocks": clocks.summary(),
         "impl": "b200",
     }
-    print(json.dumps(line), flush=True)
+    print(json.dumps(_nan_to_null(line)), flush=True)
+
+
+def _nan_to_null(x):
+    """Phases left out with --only have no number: report null rather than NaN (not JSON)."""
+    if isinstance(x, float) and math.isnan(x):
+        return None
+    if isinstance(x, dict):
+        return {k: _nan_to_null(v) for k, v in x.items()}
+    if isinstance(x, list):
+        return [_nan_to_null(v) for v in x]
+    return x
 
 
 # ----------------------------------------------------------------------------- CPU oracle
@@ -593,7 +604,7 @@ def run_reference(args):
                          "sample": f"{rows} random causal rows per step (fp64 oracle, materialised rows)"},
         "e2e": {"value": round(val, 6), "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
-    print(json.dumps(line), flush=True)
+    print(json.dumps(_nan_to_null(line)), flush=True)
 
 
 def main():
