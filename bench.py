@@ -45,6 +45,7 @@ FALLBACK_BF16_TFLOPS = 1590.0
 FWD = si.WORKLOADS["gqa_causal_8k"]
 DEC = si.WORKLOADS["decode_split_kv"]
 PAGED = si.WORKLOADS["decode_paged_ragged"]
+MHA2K = si.WORKLOADS["mha_causal_2k"]
 DOUT_ID = 9  # stream id of the backward's upstream gradient
 
 
@@ -243,6 +244,7 @@ def run_device(args):
     do_paged = args.only in ("all", "paged")
     do_bwd = args.only in ("all", "bwd")
     do_fp8 = args.only in ("all", "fp8")
+    do_tf32 = args.only in ("all", "tf32")
     if do_bwd:
         h_do_f = torch.from_numpy(inputs("fwd", seed, DOUT_ID, (B, N, Hq, d))).to(torch.bfloat16)
         b_do = h_do_f.to(dev)
@@ -295,6 +297,20 @@ def run_device(args):
         f8_ws_bytes = fa.fa_fwd_fp8_workspace_size(B, Hkv, N, d)
         f8_ws = torch.empty(f8_ws_bytes, dtype=torch.uint8, device=dev)
 
+    if do_tf32:
+        wt = MHA2K
+        tB, tN, tH, td = wt["B"], wt["N"], wt["Hq"], wt["d"]
+        tq, tk, tv = (torch.from_numpy(inputs("tf32", wt["seed"] + 100000 * rank, tid, (tB, tN, tH, td)))
+                      .to(dev) for tid in (si.Q, si.K, si.V))
+        t_o = torch.empty((tB, tN, tH, td), dtype=torch.float32, device=dev)
+        t_lse = torch.empty((tB, tH, tN), dtype=torch.float32, device=dev)
+        t_ws_bytes = fa.fa_fwd_workspace_size(tB, tH, tH, tN, tN, td, fa.FA_TF32, False)
+        t_ws = torch.empty(t_ws_bytes, dtype=torch.uint8, device=dev)
+
+    def call_tf32():
+        fa.fa_fwd(tq, tk, tv, t_o, t_lse, tB, tH, tH, tN, tN, td, 1.0 / math.sqrt(td), 1, None, fa.FA_TF32, t_ws,
+                  t_ws_bytes, st)
+
     def call_fp8():
         fa.fa_fwd_fp8(f8_q, f8_k, f8_v, f8_o, f8_lse, B, Hq, Hkv, N, N, d, scale, f8_desc[0], f8_desc[1], f8_desc[2],
                       1, f8_ws, f8_ws_bytes, st)
@@ -341,6 +357,7 @@ def run_device(args):
         call_fwd()  # the backward consumes the forward's o and lse
     bwd_ms = timed_launches(call_bwd, args.steps, args.warmup) if do_bwd else [float("nan")]
     fp8_ms = timed_launches(call_fp8, args.steps, args.warmup) if do_fp8 else [float("nan")]
+    tf32_ms = timed_launches(call_tf32, args.steps, args.warmup) if do_tf32 else [float("nan")]
     if fa.fa_last_device_error(st) != fa.FA_OK:
         raise RuntimeError("device-side timeout recorded during the benchmark")
 
@@ -386,6 +403,7 @@ def run_device(args):
     paged_mean = max_over_ranks(sum(paged_ms) / len(paged_ms), dev)
     bwd_mean = max_over_ranks(sum(bwd_ms) / len(bwd_ms), dev)
     fp8_mean = max_over_ranks(sum(fp8_ms) / len(fp8_ms), dev)
+    tf32_mean = max_over_ranks(sum(tf32_ms) / len(tf32_ms), dev)
     fwd_e2e_ms = max_over_ranks(fwd_e2e_ms, dev)
     dec_e2e_ms = max_over_ranks(dec_e2e_ms, dev)
     if world > 1:
@@ -411,6 +429,9 @@ def run_device(args):
     bwd_peak = peaks["bf16"] if (args.steps * bwd_mean) < 1000.0 else peaks["bf16_sustained"]
     fp8_tflops = F / (fp8_mean * 1e-3) / 1e12
     fp8_peak = 2.0 * (peaks["bf16"] if (args.steps * fp8_mean) < 1000.0 else peaks["bf16_sustained"])
+    F2k = fwd_flops(MHA2K)
+    tf32_tflops = F2k / (tf32_mean * 1e-3) / 1e12
+    tf32_peak = peaks["bf16"] * 1100.0 / 2250.0
     pkv = paged_kv_bytes(p_len)
     paged_gbs = pkv / (paged_mean * 1e-3) / 1e9
     cpu = cpu_baseline_fwd(args.cpu_seconds) if not args.no_cpu else None
@@ -471,6 +492,14 @@ def run_device(args):
                                      "traffic": ncu_traffic("fa_fwd_fp8/gqa_causal_8k"),
                                      "kernels": "transpose_v_e4m3_kernel + fa_fwd_kernel<128,false,fp8>",
                                      "algorithmic_flops_per_launch": F}},
+        "forward_tf32": {"value": round(aggregate_rate(F2k, world, tf32_mean) / 1e12, 2), "unit": "TFLOP/s",
+                         "ms": round(tf32_mean, 4),
+                         "workload": "mha_causal_2k (B=2, H=12, N=2048, d=64, causal) with fp32 q, k, v on the tf32 path",
+                         "roofline": {"bound": "tensor", "achieved": round(tf32_tflops, 2), "peak": round(tf32_peak, 1),
+                                      "unit": "TFLOP/s", "frac": round(tf32_tflops / tf32_peak, 4),
+                                      "peak_kind": f"measured bf16 x 1100/2250 (nominal tf32/bf16 ratio; {peaks['source']})",
+                                      "kernels": "round_tf32_kernel x2 + transpose_v_f32_kernel + fa_fwd_kernel<64,true,tf32>",
+                                      "algorithmic_flops_per_launch": F2k}},
         "backward": {"value": round(aggregate_rate(bwd_flops, world, bwd_mean) / 1e12, 2), "unit": "TFLOP/s",
                      "ms": round(bwd_mean, 4),
                      "workload": "gqa_causal_8k backward (dQ, dK, dV from the forward's O and lse; dO seeded N(0,1))",
@@ -484,7 +513,7 @@ def run_device(args):
         "e2e": {"value": round(world * F / (fwd_e2e_ms * 1e-3) / 1e12, 2), "unit": "TFLOP/s",
                 "h2d_bytes_per_step": h2d_fwd, "d2h_bytes_per_step": d2h_fwd},
         "cpu_baseline": cpu,
-        "gpu_launches": args.steps * (int(do_fwd) * 1 + int(do_dec) * 2 + int(do_paged) * 1 + int(do_bwd) * 3 + int(do_fp8) * 2)
+        "gpu_launches": args.steps * (int(do_fwd) * 1 + int(do_dec) * 2 + int(do_paged) * 1 + int(do_bwd) * 3 + int(do_fp8) * 2 + int(do_tf32) * 4)
         + (0 if args.no_e2e else e2e_steps * (int(do_fwd) * 1 + int(do_dec) * 2)),
         "clocks": clocks.summary(),
         "impl": "b200",
@@ -616,7 +645,7 @@ def main():
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--no-cpu", action="store_true", help="skip the CPU oracle baseline")
     ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer end-to-end phases")
-    ap.add_argument("--only", default="all", choices=["all", "fwd", "dec", "paged", "bwd", "fp8"],
+    ap.add_argument("--only", default="all", choices=["all", "fwd", "dec", "paged", "bwd", "fp8", "tf32"],
                     help="profiling: run one kernel family")
     args = ap.parse_args()
     if args.warmup < 3:

@@ -15,7 +15,7 @@ PKG = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(PKG, "libfa.so")
 
 FA_OK, FA_ERR_INVALID_ARG, FA_ERR_UNSUPPORTED, FA_ERR_WORKSPACE, FA_ERR_CUDA, FA_ERR_TIMEOUT = range(6)
-FA_BF16, FA_F32 = 0, 1
+FA_BF16, FA_F32, FA_TF32 = 0, 1, 2
 
 EXPORTED = ("fa_fwd", "fa_fwd_workspace_size", "fa_decode", "fa_decode_workspace_size", "fa_decode_noalloc",
             "fa_decode_paged", "fa_decode_paged_workspace_size", "fa_bwd", "fa_bwd_workspace_size", "fa_fwd_qkvpacked",
@@ -191,7 +191,8 @@ def fa_device_sm_count() -> int:
 
 
 # ------------------------------------------------------------------ tensor-level helpers
-def forward(q, k, v, causal=False, scale=None, cu_seqlens=None, out=None, lse=None, workspace=None, stream=None):
+def forward(q, k, v, causal=False, scale=None, cu_seqlens=None, out=None, lse=None, workspace=None, stream=None,
+            tf32=False):
     """O, lse for q [B,Nq,Hq,d] / k,v [B,Nk,Hkv,d] (or packed [total,H,d] with cu_seqlens).
 
     bf16 inputs give bf16 O; fp32 inputs (fixed length) are rounded to bf16 on the device and
@@ -207,11 +208,11 @@ def forward(q, k, v, causal=False, scale=None, cu_seqlens=None, out=None, lse=No
         B, Nq, Hq, d = q.shape
         Nk, Hkv = k.shape[1], k.shape[2]
         lse_shape = (B, Hq, Nq)
-    in_dtype = FA_F32 if q.dtype == torch.float32 else FA_BF16
+    in_dtype = (FA_TF32 if tf32 else FA_F32) if q.dtype == torch.float32 else FA_BF16
     if scale is None:
         scale = d ** -0.5
     if out is None:
-        out = torch.empty(q.shape, dtype=torch.float32 if in_dtype == FA_F32 else torch.bfloat16, device=q.device)
+        out = torch.empty(q.shape, dtype=torch.bfloat16 if in_dtype == FA_BF16 else torch.float32, device=q.device)
     if lse is None:
         lse = torch.empty(lse_shape, dtype=torch.float32, device=q.device)
     ws_bytes = fa_fwd_workspace_size(B, Hq, Hkv, Nq, Nk, d, in_dtype, varlen)

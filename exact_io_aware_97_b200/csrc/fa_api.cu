@@ -54,6 +54,41 @@ __global__ void __launch_bounds__(256) transpose_v_e4m3_kernel(const uint8_t* __
   }
 }
 
+// fp32 -> the nearest tf32 value (10 mantissa bits, ties to even), kept in fp32 storage.
+// Integer rounding on the bit pattern; infinities and NaN pass through.
+__device__ __forceinline__ float round_tf32(float x) {
+  uint32_t u = __float_as_uint(x);
+  if ((u & 0x7F800000u) != 0x7F800000u) {
+    u += 0x0FFFu + ((u >> 13) & 1u);
+    u &= ~0x1FFFu;
+  }
+  return __uint_as_float(u);
+}
+
+__global__ void round_tf32_kernel(const float* __restrict__ src, float* __restrict__ dst, size_t n) {
+  const size_t stride = (size_t)gridDim.x * blockDim.x;
+  for (size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += stride) dst[i] = round_tf32(src[i]);
+}
+
+// V^T for the tf32 forward (d = 64, fp32, rounded to tf32): vt[(b*Hkv + h)*64 + c][n] =
+// v[b][n][h][c] for n < Nk, 0 up to NkPad.  One block per (32-key chunk, head, sequence).
+__global__ void __launch_bounds__(256) transpose_v_f32_kernel(const float* __restrict__ v, float* __restrict__ vt,
+                                                              int Nk, int Hkv, int NkPad) {
+  __shared__ float tile[32][65];
+  const int n0 = blockIdx.x * 32, h = blockIdx.y, b = blockIdx.z;
+  for (int idx = threadIdx.x; idx < 32 * 64; idx += 256) {
+    const int r = idx >> 6, c = idx & 63;
+    const int n = n0 + r;
+    tile[r][c] = (n < Nk) ? round_tf32(v[(((size_t)b * Nk + n) * Hkv + h) * 64 + c]) : 0.f;
+  }
+  __syncthreads();
+  for (int idx = threadIdx.x; idx < 64 * 32; idx += 256) {
+    const int c = idx >> 5, r = idx & 31;
+    const int n = n0 + r;
+    if (n < NkPad) vt[(((size_t)b * Hkv + h) * 64 + c) * NkPad + n] = tile[r][c];
+  }
+}
+
 namespace {
 
 using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
@@ -98,6 +133,17 @@ bool make_map_u8(CUtensorMap* map, const void* base, const cuuint64_t (&dims)[3]
   if (!enc) return false;
   cuuint32_t estr[3] = {1, 1, 1};
   return enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void*>(base), dims, strides, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// fp32 tensor of three dimensions with the 128-byte swizzle (box inner extent 32 elements).
+bool make_map_f32(CUtensorMap* map, const void* base, const cuuint64_t (&dims)[3], const cuuint64_t (&strides)[2],
+                  const cuuint32_t (&box)[3]) {
+  EncodeTiledFn enc = get_encode_fn();
+  if (!enc) return false;
+  cuuint32_t estr[3] = {1, 1, 1};
+  return enc(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, const_cast<void*>(base), dims, strides, box, estr,
              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
@@ -219,11 +265,88 @@ const char* fa_status_string(fa_status s) {
 int fa_device_sm_count(void) { return sm_count_cached(); }
 
 size_t fa_fwd_workspace_size(int B, int Hq, int Hkv, int Nq, int Nk, int d, fa_dtype in_dtype, int varlen) {
+  if (in_dtype == FA_TF32) {
+    // tf32-rounded copies of q and k, then the rounded, transposed v
+    if (varlen || B <= 0 || Hq <= 0 || Hkv <= 0 || Nq < 0 || Nk < 0 || d != 64) return 0;
+    const size_t pad = (size_t)(Nk + 3) / 4 * 4;
+    return align_up((size_t)B * Nq * Hq * d * 4, 256) + align_up((size_t)B * Nk * Hkv * d * 4, 256) +
+           align_up((size_t)B * Hkv * d * pad * 4, 256);
+  }
   if (in_dtype != FA_F32 || varlen) return 0;
   if (B <= 0 || Hq <= 0 || Hkv <= 0 || Nq < 0 || Nk < 0 || d <= 0) return 0;
   const size_t nq = (size_t)B * Nq * Hq * d, nk = (size_t)B * Nk * Hkv * d;
   return align_up(nq * 2, 256) + 2 * align_up(nk * 2, 256);
 }
+
+}  // extern "C"
+
+namespace fa {
+namespace {
+
+// fp32 q, k, v (d = 64, fixed length) on the tf32 tensor-core path; O written as fp32.
+fa_status fwd_tf32(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq, int Hkv, int Nq,
+                   int Nk, float scale, int causal, void* workspace, size_t workspace_bytes, cudaStream_t st) {
+  constexpr int D = 64;
+  const int64_t rows_q = (int64_t)B * Nq, rows_k = (int64_t)B * Nk;
+  const int pad = (Nk + 3) / 4 * 4;
+  const size_t need = fa_fwd_workspace_size(B, Hq, Hkv, Nq, Nk, D, FA_TF32, 0);
+  if (need > 0 && (!workspace || workspace_bytes < need || !aligned16(workspace))) return FA_ERR_WORKSPACE;
+  if (B > 65535 || Hkv > 65535) return FA_ERR_UNSUPPORTED;
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  const size_t nq = (size_t)rows_q * Hq * D, nk = (size_t)rows_k * Hkv * D;
+  float* qr = reinterpret_cast<float*>(ws);
+  float* kr = reinterpret_cast<float*>(ws + align_up(nq * 4, 256));
+  float* vt = reinterpret_cast<float*>(ws + align_up(nq * 4, 256) + align_up(nk * 4, 256));
+  const int sms0 = std::max(sm_count_cached(), 1);
+  round_tf32_kernel<<<sms0 * 4, 256, 0, st>>>(static_cast<const float*>(q), qr, nq);
+  if (Nk > 0) {
+    round_tf32_kernel<<<sms0 * 4, 256, 0, st>>>(static_cast<const float*>(k), kr, nk);
+    dim3 g((pad + 31) / 32, Hkv, B);
+    transpose_v_f32_kernel<<<g, 256, 0, st>>>(static_cast<const float*>(v), vt, Nk, Hkv, pad);
+  }
+  if (cudaGetLastError() != cudaSuccess) return FA_ERR_CUDA;
+  FwdParams prm{};
+  prm.o = o;
+  prm.lse = lse;
+  prm.cu = nullptr;
+  prm.B = B;
+  prm.Hq = Hq;
+  prm.Hkv = Hkv;
+  prm.G = Hq / Hkv;
+  prm.Nq = Nq;
+  prm.Nk = Nk;
+  prm.causal = causal ? 1 : 0;
+  prm.tau = (float)((double)scale * 1.4426950408889634074);
+  prm.o_scale = 1.f;
+  prm.T = (Nq + kUnitRows - 1) / kUnitRows;
+  const int64_t units64 = (int64_t)prm.T * B * Hq;
+  if (units64 >= (int64_t(1) << 31)) return FA_ERR_UNSUPPORTED;
+  CUtensorMap mq, mk, mv;
+  const cuuint64_t dq3[3] = {D, (cuuint64_t)Hq, (cuuint64_t)rows_q};
+  const cuuint64_t sq2[2] = {D * 4, (cuuint64_t)Hq * D * 4};
+  const cuuint64_t dk3[3] = {D, (cuuint64_t)Hkv, (cuuint64_t)std::max<int64_t>(rows_k, 1)};
+  const cuuint64_t sk2[2] = {D * 4, (cuuint64_t)Hkv * D * 4};
+  const int vp = std::max(pad, 4);
+  const cuuint64_t dv3[3] = {(cuuint64_t)vp, D, (cuuint64_t)B * Hkv};
+  const cuuint64_t sv2[2] = {(cuuint64_t)vp * 4, (cuuint64_t)vp * 4 * D};
+  const cuuint32_t box_rows[3] = {32, 1, (cuuint32_t)kBM};
+  const cuuint32_t box_vt[3] = {32, D, 1};
+  if (!make_map_f32(&mq, qr, dq3, sq2, box_rows) || !make_map_f32(&mk, Nk > 0 ? kr : qr, dk3, sk2, box_rows) ||
+      !make_map_f32(&mv, Nk > 0 ? (const void*)vt : qr, dv3, sv2, box_vt))
+    return FA_ERR_CUDA;
+  auto kern = fa_fwd_kernel<D, true, kKindTF32>;
+  const int smem = FwdCfg<D, kKindTF32>::kSmemBytes;
+  if (set_smem(kern, smem) != cudaSuccess) return FA_ERR_CUDA;
+  const int sms = sm_count_cached();
+  if (sms <= 0) return FA_ERR_CUDA;
+  kern<<<std::min((int)units64, sms), kFwdThreads, smem, st>>>(mq, mk, mv, prm);
+  return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+}
+
+}  // namespace
+}  // namespace fa
+
+extern "C" {
 
 fa_status fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq, int Hkv, int Nq,
                  int Nk, int d, float scale, int causal, const int32_t* cu_seqlens, fa_dtype in_dtype,
@@ -232,9 +355,10 @@ fa_status fa_fwd(const void* q, const void* k, const void* v, void* o, float* ls
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o)) return FA_ERR_INVALID_ARG;
   if (B < 0 || Hq <= 0 || Hkv <= 0 || Nq < 0 || Nk < 0) return FA_ERR_INVALID_ARG;
   if (!(scale > 0.f) || !std::isfinite(scale)) return FA_ERR_INVALID_ARG;
-  if (in_dtype != FA_BF16 && in_dtype != FA_F32) return FA_ERR_INVALID_ARG;
+  if (in_dtype != FA_BF16 && in_dtype != FA_F32 && in_dtype != FA_TF32) return FA_ERR_INVALID_ARG;
   if (Hq % Hkv != 0) return FA_ERR_UNSUPPORTED;
   if (d != 64 && d != 128) return FA_ERR_UNSUPPORTED;
+  if (in_dtype == FA_TF32 && (d != 64 || cu_seqlens != nullptr)) return FA_ERR_UNSUPPORTED;
   const bool varlen = cu_seqlens != nullptr;
   if (varlen) {
     if (Nq != Nk) return FA_ERR_INVALID_ARG;
@@ -248,6 +372,8 @@ fa_status fa_fwd(const void* q, const void* k, const void* v, void* o, float* ls
   if (B == 0 || Nq == 0) return FA_OK;
 
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (in_dtype == FA_TF32) return fwd_tf32(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, scale, causal, workspace,
+                                           workspace_bytes, st);
   const void *qb = q, *kb = k, *vb = v;
   if (in_dtype == FA_F32) {
     const size_t need = fa_fwd_workspace_size(B, Hq, Hkv, Nq, Nk, d, in_dtype, 0);
@@ -354,8 +480,8 @@ fa_status fa_fwd_fp8(const void* q, const void* k, const void* v, void* o, float
   if (!make_map_u8(&mq, q, dq3, sq2, box_rows) || !make_map_u8(&mk, k, dk3, sk2, box_rows) ||
       !make_map_u8(&mv, Nk > 0 ? (const void*)vt : k, dv3, sv2, box_vt))
     return FA_ERR_CUDA;
-  auto kern = fa_fwd_kernel<128, false, true>;
-  const int smem = FwdCfg<128, true>::kSmemBytes;
+  auto kern = fa_fwd_kernel<128, false, kKindFP8>;
+  const int smem = FwdCfg<128, kKindFP8>::kSmemBytes;
   if (set_smem(kern, smem) != cudaSuccess) return FA_ERR_CUDA;
   const int sms = sm_count_cached();
   if (sms <= 0) return FA_ERR_CUDA;

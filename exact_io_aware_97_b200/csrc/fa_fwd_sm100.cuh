@@ -63,16 +63,21 @@ constexpr float kRescaleThreshold = 8.0f;
 constexpr uint32_t kEmuPairMask = 0x00;
 constexpr uint32_t kIntPackPairMask = 0x00;
 
-// FP8: q, k, v in e4m3 (d = 128 only), the S and P V products on the kind::f8f6f4 tensor-core
-// path with P rounded to e4m3, V read from a [d, keys] transposed copy so that both operands
-// of P V are K-major.
-template <int D, bool FP8 = false>
+// Operand kinds of the forward: bf16 (kind::f16); FP8: q, k, v in e4m3 (d = 128 only), the
+// S and P V products on the kind::f8f6f4 tensor-core path with P rounded to e4m3; TF32: fp32
+// q, k, v (d = 64 only) on the kind::tf32 path with P kept in fp32 (read as tf32).  FP8 and
+// TF32 read V from a [d, keys] transposed copy so that both operands of P V are K-major.
+constexpr int kKindBF16 = 0, kKindFP8 = 1, kKindTF32 = 2;
+
+template <int D, int KIND = kKindBF16>
 struct FwdCfg {
-  static constexpr int kTileBytes = kBM * D * (FP8 ? 1 : 2);  // one 128 x D tile
-  static constexpr int kChunkBytes = kBM * 128;                // one 128-row x 128-byte swizzle panel
+  static constexpr int kElemBytes = KIND == kKindFP8 ? 1 : (KIND == kKindTF32 ? 4 : 2);
+  static constexpr int kTileBytes = kBM * D * kElemBytes;  // one 128 x D tile
+  static constexpr int kChunkBytes = kBM * 128;            // one 128-row x 128-byte swizzle panel
   static constexpr int kPanels = kTileBytes / kChunkBytes;
-  static constexpr int kPanelCols = FP8 ? 128 : 64;            // elements per 128-byte panel row
-  static constexpr int kStages = (FP8 || D == 64) ? 8 : 4;
+  static constexpr int kPanelCols = 128 / kElemBytes;      // elements per 128-byte panel row
+  static constexpr int kVtPanelBytes = D * 128;            // V^T tile: D rows x 128 bytes of keys
+  static constexpr int kStages = KIND == kKindTF32 ? 4 : ((KIND == kKindFP8 || D == 64) ? 8 : 4);
   static constexpr int kQBytes = 2 * kTileBytes;
   static constexpr int kRingBytes = kStages * kTileBytes;
   static constexpr int kNumBars = 2 + 2 * kStages + 10;
@@ -172,12 +177,14 @@ struct UnitIter {
   }
 };
 
-template <int D, bool OUT_F32, bool FP8 = false>
+template <int D, bool OUT_F32, int KIND = kKindBF16>
 __global__ void __launch_bounds__(kFwdThreads, 1)
     fa_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                   const __grid_constant__ CUtensorMap tmV, const FwdParams p) {
+  constexpr bool FP8 = KIND == kKindFP8, TF32 = KIND == kKindTF32;
   static_assert(!FP8 || (D == 128 && !OUT_F32), "fp8 forward: d = 128, bf16 output");
-  using C = FwdCfg<D, FP8>;
+  static_assert(!TF32 || (D == 64 && OUT_F32), "tf32 forward: d = 64, fp32 output");
+  using C = FwdCfg<D, KIND>;
   constexpr int NS = C::kStages;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -305,10 +312,13 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
               break;
             }
             mbar_arrive_expect_tx_elect(full + slot, C::kTileBytes);
-            if (FP8 && kv) {
-              // V^T tile: d rows of 128 keys from the [B * Hkv, d, keys] transposed copy
-              tma_load_3d_hint_elect(sRing + slot * C::kTileBytes, &tmV, j * kBN, 0, un.b * p.Hkv + un.kvh,
-                                     full + slot, kv_policy);
+            if ((FP8 || TF32) && kv) {
+              // V^T tile: d rows of 128 keys from the [B * Hkv, d, keys] transposed copy, in
+              // 128-byte panels of keys (one for e4m3, four for fp32)
+              for (int c = 0; c < C::kTileBytes / C::kVtPanelBytes; ++c)
+                tma_load_3d_hint_elect(sRing + slot * C::kTileBytes + c * C::kVtPanelBytes, &tmV,
+                                       j * kBN + c * C::kPanelCols, 0, un.b * p.Hkv + un.kvh, full + slot,
+                                       kv_policy);
             } else {
               for (int c = 0; c < C::kPanels; ++c)
                 tma_load_3d_hint_elect(sRing + slot * C::kTileBytes + c * C::kChunkBytes, kv ? &tmV : &tmK,
@@ -324,8 +334,9 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
   } else if (warp == 8) {
     // ================================================================ MMA issuer
     {
-      constexpr uint32_t idS = FP8 ? idesc_e4m3_f32(kBM, kBN) : idesc_bf16_f32(kBM, kBN, false);
-      constexpr uint32_t idPV = FP8 ? idesc_e4m3_f32(kBM, D) : idesc_bf16_f32(kBM, D, true);
+      constexpr uint32_t idS = FP8 ? idesc_e4m3_f32(kBM, kBN)
+                                   : (TF32 ? idesc_tf32_f32(kBM, kBN) : idesc_bf16_f32(kBM, kBN, false));
+      constexpr uint32_t idPV = FP8 ? idesc_e4m3_f32(kBM, D) : (TF32 ? idesc_tf32_f32(kBM, D) : idesc_bf16_f32(kBM, D, true));
       const uint32_t qbase = smem_u32(sQ);
       const uint32_t rbase = smem_u32(sRing);
       uint32_t g = 0, qcount = 0;
@@ -334,15 +345,17 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       UnitWalker wk;
       bool ok = true;
 
-      // k-steps of 32 bytes along d (16 bf16 or 32 e4m3 elements), four per 128-byte panel
+      // k-steps of 32 bytes along d (16 bf16, 32 e4m3 or 8 tf32 elements), four per panel
       auto issue_S = [&](int i, uint32_t slot) {
 #pragma unroll
-        for (int kk = 0; kk < D * (FP8 ? 1 : 2) / 32; ++kk) {
+        for (int kk = 0; kk < D * C::kElemBytes / 32; ++kk) {
           const uint32_t off = (kk >> 2) * C::kChunkBytes + (kk & 3) * 32;
           const uint64_t a = smem_desc_sw128(qbase + i * C::kTileBytes + off, 16, 1024);
           const uint64_t bd = smem_desc_sw128(rbase + slot * C::kTileBytes + off, 16, 1024);
           if (FP8)
             umma_ss_f8_elect(tmem + i * kBN, a, bd, idS, kk > 0 ? 1u : 0u);
+          else if (TF32)
+            umma_ss_tf32_elect(tmem + i * kBN, a, bd, idS, kk > 0 ? 1u : 0u);
           else
             umma_ss_elect(tmem + i * kBN, a, bd, idS, kk > 0 ? 1u : 0u);
         }
@@ -350,7 +363,16 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       // O_i (+)= P_i V for the keys of one half (8 k-steps of 16 keys in all).
       // (P in TMEM: 8 columns per k-step either way, 16 keys of bf16 or 32 keys of e4m3)
       auto issue_PV_half = [&](int i, uint32_t slot, int half, bool acc) {
-        if (FP8) {
+        if (TF32) {
+          // P in fp32 over all 128 columns of S; k-steps of 8 keys (32 bytes of a V^T row)
+#pragma unroll
+          for (int k8 = 0; k8 < kBN / 16; ++k8) {
+            const int kk = half * (kBN / 16) + k8;
+            const uint64_t bd =
+                smem_desc_sw128(rbase + slot * C::kTileBytes + (kk >> 2) * C::kVtPanelBytes + (kk & 3) * 32, 16, 1024);
+            umma_ts_tf32_elect(tmem + C::kColO + i * D, tmem + i * kBN + kk * 8, bd, idPV, (acc || kk > 0) ? 1u : 0u);
+          }
+        } else if (FP8) {
 #pragma unroll
           for (int k2 = 0; k2 < kBN / 64; ++k2) {
             const int kk = half * (kBN / 64) + k2;  // 32 keys = 32 bytes of each V^T row
@@ -524,7 +546,22 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         uint64_t lsum[2] = {f2(0.f, 0.f), f2(0.f, 0.f)};
 #pragma unroll
         for (int half = 0; half < 2; ++half) {
-          if (FP8) {
+          if (TF32) {
+            // fp32 P over the S columns of its own keys (read by the tensor core as tf32)
+            uint32_t pk[2][32];
+#pragma unroll
+            for (int e = 0; e < 32; ++e) {
+              const int g = 32 * half + e;  // column pair
+              float x0, x1;
+              f2_split(f2_fma(f2(s[2 * g], s[2 * g + 1]), tau2, nms2), x0, x1);
+              const float p0 = ex2_approx(x0), p1 = ex2_approx(x1);
+              lsum[g & 1] = f2_add(lsum[g & 1], f2(p0, p1));
+              pk[e >> 4][2 * (e & 15)] = __float_as_uint(p0);
+              pk[e >> 4][2 * (e & 15) + 1] = __float_as_uint(p1);
+            }
+            tmem_st32(tS + 64 * half, pk[0]);
+            tmem_st32(tS + 64 * half + 32, pk[1]);
+          } else if (FP8) {
             // e4m3 P, four keys per TMEM column: 64 keys in 16 columns
             uint32_t pk[16];
 #pragma unroll

@@ -55,7 +55,7 @@ typedef enum {
   FA_ERR_TIMEOUT = 5      /* a device wait gave up (reported by fa_last_device_error) */
 } fa_status;
 
-typedef enum { FA_BF16 = 0, FA_F32 = 1 } fa_dtype;
+typedef enum { FA_BF16 = 0, FA_F32 = 1, FA_TF32 = 2 } fa_dtype;
 
 /* Forward attention.
  *
@@ -68,7 +68,10 @@ typedef enum { FA_BF16 = 0, FA_F32 = 1 } fa_dtype;
  *   on the device only).  B <= 1024.
  *
  * in_dtype FA_BF16: q, k, v, o are bf16.  FA_F32: q, k, v are fp32, rounded to bf16 (nearest
- *   even) into the workspace first, and o is written as fp32; fixed length only.
+ *   even) into the workspace first, and o is written as fp32; fixed length only.  FA_TF32: q, k,
+ *   v are fp32, rounded to tf32 (10 mantissa bits, nearest even) into the workspace, and the
+ *   products run on the tf32 tensor-core path with P kept in fp32; o fp32; fixed length,
+ *   d = 64 (the workspace also holds v transposed).
  * Accumulation is fp32; P is rounded to bf16 before the P*V product.
  * scale: the score multiplier, > 0 (1/sqrt(d) in "LLM basics", chapter 1 section 3).
  * causal: query i of a sequence with nq queries and nk keys sees keys j <= i + nk - nq

@@ -78,6 +78,14 @@ def round_bf16(x32: np.ndarray) -> np.ndarray:
     return r.view(np.float32)
 
 
+def round_tf32(x32: np.ndarray) -> np.ndarray:
+    """Round float32 values to tf32 (10 mantissa bits, nearest even), returned as float32."""
+    u = np.ascontiguousarray(x32, dtype=np.float32).view(np.uint32).astype(np.uint64)
+    finite = (u & 0x7F800000) != 0x7F800000
+    r = (u + 0x0FFF + ((u >> 13) & 1)) & ~np.uint64(0x1FFF)
+    return np.where(finite, r, u).astype(np.uint32).view(np.float32)
+
+
 def normal(seed: int, tensor_id: int, shape, dtype: str = "bf16", threads: int | None = None) -> np.ndarray:
     """N(0,1) tensor of `shape` stored as `dtype` ('bf16' or 'f32'), as float32 values."""
     n = int(np.prod(shape))

@@ -21,3 +21,11 @@ def test_e4m3_rounds_to_nearest_even():
     vals = np.array([448.0, 1.0625, 1.1875, 1.07], dtype=np.float32)
     _, deq, _ = si.to_e4m3(vals)
     assert deq[1:].tolist() == [1.0, 1.25, 1.125]
+
+
+def test_tf32_rounding_to_nearest_even():
+    # 1 + 2^-10 is a tf32 value; 1 + 2^-11 is the midpoint between 1 and it (ties to even: 1),
+    # 1 + 3 * 2^-11 is the midpoint between 1 + 2^-10 and 1 + 2^-9 (ties to even: 1 + 2^-9)
+    x = np.array([1 + 2.0 ** -10, 1 + 2.0 ** -11, 1 + 3 * 2.0 ** -11, 1 + 2.0 ** -11 + 2.0 ** -20, -3.0],
+                 dtype=np.float32)
+    assert si.round_tf32(x).tolist() == [1 + 2.0 ** -10, 1.0, 1 + 2.0 ** -9, 1 + 2.0 ** -10, -3.0]
