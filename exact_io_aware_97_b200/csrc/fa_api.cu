@@ -231,11 +231,21 @@ fa_status launch_bwd(const void* q, const void* k, const void* v, const BwdParam
   if (pre_blocks > 0) fa_bwd_pre_kernel<D><<<pre_blocks, 256, 0, st>>>(prm);
   if (cudaGetLastError() != cudaSuccess) return FA_ERR_CUDA;
   if (prm.Nk > 0) {
-    auto kern = fa_bwd_kernel<D>;
-    const int smem = BwdCfg<D>::kSmemBytes;
-    if (set_smem(kern, smem) != cudaSuccess) return FA_ERR_CUDA;
     dim3 grid((prm.Nk + kBwdTile - 1) / kBwdTile, prm.Hkv, prm.B);
-    kern<<<grid, kBwdThreads, smem, st>>>(mq, mk, mv, mdo, prm);
+    if (D == 128) {
+      // pairs of 64 queries, two in flight: Q and dO maps with 64-row boxes
+      CUtensorMap mq64, mdo64;
+      if (!make_map(&mq64, q, D, prm.Hq, rows_q, kBwdQ) || !make_map(&mdo64, prm.dout, D, prm.Hq, rows_q, kBwdQ))
+        return FA_ERR_CUDA;
+      const int smem = Bwd2Cfg::kSmemBytes;
+      if (set_smem(fa_bwd2_kernel, smem) != cudaSuccess) return FA_ERR_CUDA;
+      fa_bwd2_kernel<<<grid, kBwdThreads, smem, st>>>(mq64, mk, mv, mdo64, prm);
+    } else {
+      auto kern = fa_bwd_kernel<D>;
+      const int smem = BwdCfg<D>::kSmemBytes;
+      if (set_smem(kern, smem) != cudaSuccess) return FA_ERR_CUDA;
+      kern<<<grid, kBwdThreads, smem, st>>>(mq, mk, mv, mdo, prm);
+    }
     if (cudaGetLastError() != cudaSuccess) return FA_ERR_CUDA;
   }
   const size_t n4 = (size_t)prm.B * prm.Nq * prm.Hq * D / 4;

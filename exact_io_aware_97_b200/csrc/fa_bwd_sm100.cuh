@@ -431,4 +431,330 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   }
 }
 
+// ------------------------------------------------------------------ main, d = 128: two pairs in flight
+//
+// Same method as fa_bwd_kernel, arranged so that the tensor core and the elementwise
+// warpgroups work on different pairs at once: pairs of 64 queries, two TMEM buffers
+//   S_b = TMEM[128 b, 128 b + 64), DP_b = TMEM[128 b + 64, 128 b + 128)   (b = pair & 1)
+// dV = TMEM[256, 384), dK = TMEM[384, 512).  Per pair t (buffer b):
+//   S^T = K Q^T -> S_b, dP^T = V dO^T -> DP_b                        (tcgen05, N = 64)
+//   elementwise: P^T (bf16) over S_b[0,32), dS^T (bf16) over S_b[32,64), dS to shared memory
+//   dV += P^T dO, dK += dS^T Q                                        (A from TMEM)
+//   dQ^T = K^T dS -> DP_b   (M = d on the TMEM lanes, so each warp's dQ read-out covers 32
+//                            consecutive d: coalesced fp32 reductions)
+// The MMA warp issues S(t) and dP(t) before the gradient products of pair t-1, so the
+// elementwise step of pair t overlaps those products; the warpgroups read dQ^T(t-1) out after
+// the elementwise step of pair t.
+constexpr int kBwdQ = 64;  // queries per pair
+constexpr int kBwdSlots = 3;
+
+struct Bwd2Cfg {
+  static constexpr int D = 128;
+  static constexpr int kKTile = kBwdTile * D * 2;       // 32 KB: 128 keys, 2 panels of 16 KB
+  static constexpr int kKPanel = kBwdTile * 128;
+  static constexpr int kQTile = kBwdQ * D * 2;          // 16 KB: 64 queries, 2 panels of 8 KB
+  static constexpr int kQPanel = kBwdQ * 128;
+  static constexpr int kDSTile = kBwdTile * kBwdQ * 2;  // 16 KB: 128 keys x 64 queries
+  static constexpr int kVecBytes = kBwdQ * 4;
+  static constexpr int kOffK = 0;
+  static constexpr int kOffV = kKTile;
+  static constexpr int kOffQ = 2 * kKTile;                          // [slots]
+  static constexpr int kOffDO = kOffQ + kBwdSlots * kQTile;         // [slots]
+  static constexpr int kOffDS = kOffDO + kBwdSlots * kQTile;        // [2]
+  static constexpr int kOffVec = kOffDS + 2 * kDSTile;              // [slots][lse2, D]
+  static constexpr int kOffBar = kOffVec + kBwdSlots * 2 * kVecBytes;
+  static constexpr int kNumBars = 24;
+  static constexpr int kUsed = kOffBar + kNumBars * 8 + 16;
+  static constexpr int kSmemBytes = kUsed + 1024;
+  static constexpr uint32_t kColDV = 256, kColDK = 384;
+};
+
+__global__ void __launch_bounds__(kBwdThreads, 1)
+    fa_bwd2_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                   const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmDO,
+                   const BwdParams p) {
+  using C = Bwd2Cfg;
+  constexpr int D = C::D;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  {
+    uint32_t dyn;
+    asm volatile("mov.u32 %0, %%dynamic_smem_size;" : "=r"(dyn));
+    if ((uint32_t)(smem - smem_raw) + (uint32_t)C::kUsed > dyn) {
+      if (threadIdx.x == 0) atomicOr(&g_error_word, kErrSmem);
+      return;
+    }
+  }
+  uint8_t* sK = smem + C::kOffK;
+  uint8_t* sV = smem + C::kOffV;
+  uint8_t* sQ = smem + C::kOffQ;
+  uint8_t* sDO = smem + C::kOffDO;
+  uint8_t* sDS = smem + C::kOffDS;
+  float* sVec = reinterpret_cast<float*>(smem + C::kOffVec);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kOffBar);
+  uint64_t* kv_full = bars + 0;
+  uint64_t* q_full = bars + 1;     // [slots]
+  uint64_t* q_empty = bars + 4;    // [slots]
+  uint64_t* sdp_full = bars + 7;   // [2]
+  uint64_t* ld_done = bars + 9;    // [2]
+  uint64_t* pds_ready = bars + 11; // [2]
+  uint64_t* dq_full = bars + 13;   // [2]
+  uint64_t* buf_free = bars + 15;  // [2]
+  uint64_t* acc_done = bars + 17;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + C::kNumBars);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int ntile = blockIdx.x, kvh = blockIdx.y, b = blockIdx.z;
+  const int n0 = ntile * kBwdTile;
+  const int diag = p.Nk - p.Nq;
+  const int nq_tiles = (p.Nq + kBwdQ - 1) / kBwdQ;
+  int i_lo = 0;
+  if (p.causal) {
+    const int need = n0 - diag - (kBwdQ - 1);  // first 64-query tile whose last query sees key n0
+    i_lo = need <= 0 ? 0 : (need + kBwdQ - 1) / kBwdQ;
+  }
+  const int ntq = max(0, nq_tiles - i_lo);
+  const int T = ntq * p.G;
+
+  if (threadIdx.x == 0) {
+    mbar_init(kv_full, 1);
+    for (int s = 0; s < kBwdSlots; ++s) {
+      mbar_init(q_full + s, 1);
+      mbar_init(q_empty + s, 1);
+    }
+    for (int x = 0; x < 2; ++x) {
+      mbar_init(sdp_full + x, 1);
+      mbar_init(ld_done + x, 8);
+      mbar_init(pds_ready + x, 8);
+      mbar_init(dq_full + x, 1);
+      mbar_init(buf_free + x, 8);
+    }
+    mbar_init(acc_done, 1);
+    fence_barrier_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0) {
+    // ============================================================ TMA producer
+    if (T > 0) {
+      mbar_arrive_expect_tx_elect(kv_full, 2 * C::kKTile);
+      for (int c = 0; c < D / 64; ++c) {
+        tma_load_3d_elect(sK + c * C::kKPanel, &tmK, c * 64, kvh, b * p.Nk + n0, kv_full);
+        tma_load_3d_elect(sV + c * C::kKPanel, &tmV, c * 64, kvh, b * p.Nk + n0, kv_full);
+      }
+      for (int t = 0; t < T; ++t) {
+        const int slot = t % kBwdSlots;
+        if (t >= kBwdSlots && !warp_wait(q_empty + slot, ((t / kBwdSlots) - 1) & 1)) break;
+        const int h = kvh * p.G + t / ntq;
+        const int q0 = (i_lo + t % ntq) * kBwdQ;
+        mbar_arrive_expect_tx_elect(q_full + slot, 2 * C::kQTile + 2 * C::kVecBytes);
+        for (int c = 0; c < D / 64; ++c) {
+          tma_load_3d_elect(sQ + slot * C::kQTile + c * C::kQPanel, &tmQ, c * 64, h, b * p.Nq + q0, q_full + slot);
+          tma_load_3d_elect(sDO + slot * C::kQTile + c * C::kQPanel, &tmDO, c * 64, h, b * p.Nq + q0,
+                            q_full + slot);
+        }
+        const size_t voff = ((size_t)b * p.Hq + h) * p.NqPad + q0;
+        bulk_load_elect(sVec + (slot * 2 + 0) * kBwdQ, p.lse2 + voff, C::kVecBytes, q_full + slot);
+        bulk_load_elect(sVec + (slot * 2 + 1) * kBwdQ, p.dvec + voff, C::kVecBytes, q_full + slot);
+      }
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    // ============================================================ MMA issuer
+    if (T > 0) {
+      constexpr uint32_t idS = idesc_bf16_f32(kBwdTile, kBwdQ, false);
+      constexpr uint32_t idAcc = idesc_bf16_f32(kBwdTile, D, true);
+      constexpr uint32_t idQ = idesc_bf16_f32_mn(D, kBwdQ, true, true);
+      const uint32_t kb = smem_u32(sK), vb = smem_u32(sV), qb = smem_u32(sQ), dob = smem_u32(sDO);
+      const uint32_t dsb = smem_u32(sDS);
+      bool ok = warp_wait(kv_full, 0);
+      tc_fence_after();
+      for (int t = 0; t <= T && ok; ++t) {
+        if (t < T) {
+          const int slot = t % kBwdSlots, bb = t & 1;
+          if (!warp_wait(q_full + slot, (t / kBwdSlots) & 1)) break;
+          if (t >= 2 && !warp_wait(buf_free + bb, ((t >> 1) - 1) & 1)) break;
+          tc_fence_after();
+          const uint32_t qs = qb + slot * C::kQTile, ds = dob + slot * C::kQTile;
+          const uint32_t cS = 128 * bb, cDP = 128 * bb + 64;
+#pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const uint32_t ka = (kk >> 2) * C::kKPanel + (kk & 3) * 32;
+            const uint32_t kq = (kk >> 2) * C::kQPanel + (kk & 3) * 32;
+            umma_ss_elect(tmem + cS, smem_desc_sw128(kb + ka, 16, 1024), smem_desc_sw128(qs + kq, 16, 1024), idS,
+                          kk > 0 ? 1u : 0u);
+          }
+#pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const uint32_t ka = (kk >> 2) * C::kKPanel + (kk & 3) * 32;
+            const uint32_t kq = (kk >> 2) * C::kQPanel + (kk & 3) * 32;
+            umma_ss_elect(tmem + cDP, smem_desc_sw128(vb + ka, 16, 1024), smem_desc_sw128(ds + kq, 16, 1024), idS,
+                          kk > 0 ? 1u : 0u);
+          }
+          umma_commit_elect(sdp_full + bb);
+        }
+        if (t >= 1) {
+          const int tp = t - 1, slot = tp % kBwdSlots, bb = tp & 1;
+          if (!warp_wait(pds_ready + bb, (tp >> 1) & 1)) break;
+          tc_fence_after();
+          const uint32_t qs = qb + slot * C::kQTile, ds = dob + slot * C::kQTile;
+          const uint32_t cS = 128 * bb, cDP = 128 * bb + 64;
+#pragma unroll
+          for (int kk = 0; kk < kBwdQ / 16; ++kk) {
+            const uint32_t acc = (tp > 0 || kk > 0) ? 1u : 0u;
+            umma_ts_elect(tmem + C::kColDV, tmem + cS + kk * 8,
+                          smem_desc_sw128(ds + kk * 16 * 128, C::kQPanel, 1024), idAcc, acc);
+            umma_ts_elect(tmem + C::kColDK, tmem + cS + 32 + kk * 8,
+                          smem_desc_sw128(qs + kk * 16 * 128, C::kQPanel, 1024), idAcc, acc);
+          }
+          // dQ^T = K^T dS: A = K (keys x d) read d-major, B = dS (keys x queries) query-major
+#pragma unroll
+          for (int kk = 0; kk < kBwdTile / 16; ++kk)
+            umma_ss_elect(tmem + cDP, smem_desc_sw128(kb + kk * 16 * 128, C::kKPanel, 1024),
+                          smem_desc_sw128(dsb + bb * C::kDSTile + kk * 16 * 128, C::kDSTile, 1024), idQ,
+                          kk > 0 ? 1u : 0u);
+          umma_commit_elect(dq_full + bb);
+          umma_commit_elect(q_empty + slot);
+        }
+      }
+      umma_commit_elect(acc_done);
+    }
+    __syncwarp();
+  } else if (warp >= 4) {
+    // ============================================================ elementwise warpgroups
+    const int wg = (warp - 4) >> 2;
+    const int r = (warp & 3) * 32 + lane;  // TMEM lane: key row (S, dP) or d (dQ^T)
+    const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
+    const int key = n0 + r;
+    const bool key_ok = key < p.Nk;
+    const float tau = p.tau;
+    bool ok = true;
+
+    auto read_dq = [&](int tp) -> bool {
+      const int bb = tp & 1;
+      if (!warp_wait(dq_full + bb, (tp >> 1) & 1)) return false;
+      tc_fence_after();
+      uint32_t a[32];
+      tmem_ld32(tmem + lane_off + 128 * bb + 64 + 32 * wg, a);
+      tmem_wait_ld();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(buf_free + bb);
+      const int h = kvh * p.G + tp / ntq;
+      const int qb0 = (i_lo + tp % ntq) * kBwdQ + 32 * wg;
+      float* base = p.dq_acc + (((size_t)b * p.Nq + qb0) * p.Hq + h) * D + r;
+      const size_t qstride = (size_t)p.Hq * D;
+#pragma unroll
+      for (int e = 0; e < 32; ++e)
+        if (qb0 + e < p.Nq) red_add_f32(base + e * qstride, __uint_as_float(a[e]));
+      return true;
+    };
+
+    for (int t = 0; t < T && ok; ++t) {
+      const int slot = t % kBwdSlots, bb = t & 1;
+      const int q0 = (i_lo + t % ntq) * kBwdQ;
+      if (!warp_wait(q_full + slot, (t / kBwdSlots) & 1) || !warp_wait(sdp_full + bb, (t >> 1) & 1)) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      const uint32_t cS = 128 * bb, cDP = 128 * bb + 64;
+      const float* l2 = sVec + (slot * 2 + 0) * kBwdQ + 32 * wg;
+      const float* dd = sVec + (slot * 2 + 1) * kBwdQ + 32 * wg;
+      uint32_t pk[16], dsk[16];
+      {
+        uint32_t sv[32], dpv[32];
+        tmem_ld32(tmem + lane_off + cS + 32 * wg, sv);
+        tmem_ld32(tmem + lane_off + cDP + 32 * wg, dpv);
+        tmem_wait_ld();
+        const int qfirst = q0 + 32 * wg;
+        int lim = 0;  // columns e < lim are masked
+        if (!key_ok) lim = 32;
+        else if (p.causal) lim = min(32, max(0, key - diag - qfirst));
+#pragma unroll
+        for (int e = 0; e < 16; ++e) {
+          const float4 lv = *reinterpret_cast<const float4*>(l2 + 4 * (e >> 1));
+          const float4 dv4 = *reinterpret_cast<const float4*>(dd + 4 * (e >> 1));
+          const float la = (e & 1) ? lv.z : lv.x, lb = (e & 1) ? lv.w : lv.y;
+          const float da = (e & 1) ? dv4.z : dv4.x, db = (e & 1) ? dv4.w : dv4.y;
+          float p0 = ex2_approx(fmaf(__uint_as_float(sv[2 * e]), tau, -la));
+          float p1 = ex2_approx(fmaf(__uint_as_float(sv[2 * e + 1]), tau, -lb));
+          if (2 * e < lim) p0 = 0.f;
+          if (2 * e + 1 < lim) p1 = 0.f;
+          pk[e] = pack_bf16x2(p0, p1);
+          dsk[e] = pack_bf16x2(p0 * (__uint_as_float(dpv[2 * e]) - da), p1 * (__uint_as_float(dpv[2 * e + 1]) - db));
+        }
+      }
+      // dS row r: 64 queries = one 128-byte row of the query-major tile; this warpgroup's 32
+      // queries are units 4 wg .. 4 wg + 3 (stored at u ^ (r % 8))
+      {
+        uint8_t* row = sDS + bb * C::kDSTile + r * 128;
+#pragma unroll
+        for (int u = 0; u < 4; ++u)
+          *reinterpret_cast<uint4*>(row + (((4 * wg + u) ^ (r & 7)) << 4)) =
+              make_uint4(dsk[4 * u], dsk[4 * u + 1], dsk[4 * u + 2], dsk[4 * u + 3]);
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(ld_done + bb);
+      if (!warp_wait(ld_done + bb, (t >> 1) & 1)) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      tmem_st16(tmem + lane_off + cS + 16 * wg, pk);
+      tmem_st16(tmem + lane_off + cS + 32 + 16 * wg, dsk);
+      tmem_wait_st();
+      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(pds_ready + bb);
+      if (t >= 1 && !read_dq(t - 1)) {
+        ok = false;
+        break;
+      }
+    }
+    if (ok && T > 0) ok = read_dq(T - 1);
+    // ---- epilogue: dV (warpgroup 0) and dK = scale * acc (warpgroup 1), rows of this key tile
+    const bool have = T > 0 && ok && warp_wait(acc_done, 0);
+    tc_fence_after();
+    __nv_bfloat16* dst = (wg ? p.dk : p.dv) + (((size_t)b * p.Nk + key) * p.Hkv + kvh) * D;
+    const float mul = wg ? p.scale : 1.f;
+#pragma unroll
+    for (int c = 0; c < D / 32; ++c) {
+      uint32_t a[32];
+      if (have) {
+        tmem_ld32(tmem + lane_off + (wg ? C::kColDK : C::kColDV) + 32 * c, a);
+        tmem_wait_ld();
+      } else {
+#pragma unroll
+        for (int e = 0; e < 32; ++e) a[e] = 0u;
+      }
+      if (key_ok) {
+        uint4* d4 = reinterpret_cast<uint4*>(dst + 32 * c);
+#pragma unroll
+        for (int e = 0; e < 4; ++e)
+          d4[e] = make_uint4(pack_bf16x2(__uint_as_float(a[8 * e]) * mul, __uint_as_float(a[8 * e + 1]) * mul),
+                             pack_bf16x2(__uint_as_float(a[8 * e + 2]) * mul, __uint_as_float(a[8 * e + 3]) * mul),
+                             pack_bf16x2(__uint_as_float(a[8 * e + 4]) * mul, __uint_as_float(a[8 * e + 5]) * mul),
+                             pack_bf16x2(__uint_as_float(a[8 * e + 6]) * mul, __uint_as_float(a[8 * e + 7]) * mul));
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
 }  // namespace fa

@@ -261,6 +261,11 @@ __device__ __forceinline__ void bulk_load_elect(void* smem_dst, const void* gsrc
       : "memory");
 }
 
+// One fp32 addition to global memory (no return value).
+__device__ __forceinline__ void red_add_f32(float* addr, float a) {
+  asm volatile("red.global.add.f32 [%0], %1;" ::"l"(addr), "f"(a) : "memory");
+}
+
 // Four fp32 additions to global memory in one reduction (no return value).
 __device__ __forceinline__ void red_add_v4(float* addr, float a, float b, float c, float d) {
   asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(addr), "f"(a), "f"(b), "f"(c), "f"(d)
