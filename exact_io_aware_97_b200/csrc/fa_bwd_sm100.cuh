@@ -673,23 +673,34 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         uint32_t sv[32], dpv[32];
         tmem_ld32(tmem + lane_off + cS + 32 * wg, sv);
         tmem_ld32(tmem + lane_off + cDP + 32 * wg, dpv);
+        // the row vectors of this warpgroup's 32 queries (broadcast reads), while TMEM loads
+        float4 lv[8], dv4[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          lv[e] = reinterpret_cast<const float4*>(l2)[e];
+          dv4[e] = reinterpret_cast<const float4*>(dd)[e];
+        }
         tmem_wait_ld();
         const int qfirst = q0 + 32 * wg;
         int lim = 0;  // columns e < lim are masked
         if (!key_ok) lim = 32;
         else if (p.causal) lim = min(32, max(0, key - diag - qfirst));
+        const uint64_t tau2 = f2(tau, tau);
 #pragma unroll
         for (int e = 0; e < 16; ++e) {
-          const float4 lv = *reinterpret_cast<const float4*>(l2 + 4 * (e >> 1));
-          const float4 dv4 = *reinterpret_cast<const float4*>(dd + 4 * (e >> 1));
-          const float la = (e & 1) ? lv.z : lv.x, lb = (e & 1) ? lv.w : lv.y;
-          const float da = (e & 1) ? dv4.z : dv4.x, db = (e & 1) ? dv4.w : dv4.y;
-          float p0 = ex2_approx(fmaf(__uint_as_float(sv[2 * e]), tau, -la));
-          float p1 = ex2_approx(fmaf(__uint_as_float(sv[2 * e + 1]), tau, -lb));
+          const float4 L = lv[e >> 1], Dv = dv4[e >> 1];
+          const uint64_t nl = (e & 1) ? f2(-L.z, -L.w) : f2(-L.x, -L.y);
+          const uint64_t nd = (e & 1) ? f2(-Dv.z, -Dv.w) : f2(-Dv.x, -Dv.y);
+          float x0, x1;
+          f2_split(f2_fma(f2(__uint_as_float(sv[2 * e]), __uint_as_float(sv[2 * e + 1])), tau2, nl), x0, x1);
+          float p0 = ex2_approx(x0), p1 = ex2_approx(x1);
           if (2 * e < lim) p0 = 0.f;
           if (2 * e + 1 < lim) p1 = 0.f;
           pk[e] = pack_bf16x2(p0, p1);
-          dsk[e] = pack_bf16x2(p0 * (__uint_as_float(dpv[2 * e]) - da), p1 * (__uint_as_float(dpv[2 * e + 1]) - db));
+          const uint64_t g2 = f2_add(f2(__uint_as_float(dpv[2 * e]), __uint_as_float(dpv[2 * e + 1])), nd);
+          float g0, g1;
+          f2_split(f2_fma(f2(p0, p1), g2, f2(0.f, 0.f)), g0, g1);
+          dsk[e] = pack_bf16x2(g0, g1);
         }
       }
       // dS row r: 64 queries = one 128-byte row of the query-major tile; this warpgroup's 32
