@@ -89,3 +89,17 @@ def test_bwd_gqa_causal_8k_one_group(orc):
     check_grad(dq[:, :, hs], rq, "dQ")
     check_grad(dk[:, :, g:g + 1], rk, "dK")
     check_grad(dv[:, :, g:g + 1], rv, "dV")
+
+
+def test_bwd_mha_causal_2k_full(orc):
+    """B=2, H=12, N=2048, d=64, causal (the pages' packed example shape): every gradient
+    element against the oracle (the d = 64 kernel)."""
+    w = si.WORKLOADS["mha_causal_2k"]
+    B, N, Hq, Hkv, d = w["B"], w["N"], w["Hq"], w["Hkv"], w["d"]
+    q, k, v, do = _inputs(w["seed"], B, N, N, Hq, Hkv, d)
+    scale = 1.0 / math.sqrt(d)
+    dq, dk, dv = _gpu_bwd(q, k, v, do, True, scale)
+    rq, rk, rv = orc.attention_bwd(q, k, v, do, scale, causal=True)
+    check_grad(dq, rq, "dQ")
+    check_grad(dk, rk, "dK")
+    check_grad(dv, rv, "dV")
