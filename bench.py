@@ -508,7 +508,7 @@ def run_device(args):
                                   "unit": "TFLOP/s", "frac": round(bwd_tflops / bwd_peak, 4),
                                   "peak_kind": f"measured ({peaks['source']})",
                                   "traffic": ncu_traffic("fa_bwd/gqa_causal_8k"),
-                                  "kernels": "fa_bwd_pre_kernel<128> + fa_bwd_kernel<128> + fa_bwd_dq_kernel<128>",
+                                  "kernels": "fa_bwd_pre_kernel<128> + fa_bwd2_kernel + fa_bwd_dq_kernel<128>",
                                   "algorithmic_flops_per_launch": bwd_flops}},
         "e2e": {"value": round(world * F / (fwd_e2e_ms * 1e-3) / 1e12, 2), "unit": "TFLOP/s",
                 "h2d_bytes_per_step": h2d_fwd, "d2h_bytes_per_step": d2h_fwd},
