@@ -142,3 +142,59 @@ def test_binding_raises_fa_error(lib):
     with pytest.raises(fa.FaError) as e:
         fa.fa_fwd(256, 256, 256, 256, None, 1, 2, 1, 8, 8, 96, 0.1, 1, stream=0)
     assert e.value.status == fa.FA_ERR_UNSUPPORTED
+
+
+def test_bwd_rejects_before_launch(lib):
+    def st(**kw):
+        a = dict(q=256, k=256, v=256, o=256, do=256, lse=512, dq=256, dk=256, dv=256, B=1, Hq=2, Hkv=1, Nq=8, Nk=8,
+                 d=128, scale=0.1, causal=1, ws=256, wsb=1 << 30)
+        a.update(kw)
+        return lib.fa_bwd(a["q"], a["k"], a["v"], a["o"], a["do"], a["lse"], a["dq"], a["dk"], a["dv"], a["B"],
+                          a["Hq"], a["Hkv"], a["Nq"], a["Nk"], a["d"], ctypes.c_float(a["scale"]), a["causal"],
+                          a["ws"], a["wsb"], None)
+    assert st(do=None) == fa.FA_ERR_INVALID_ARG
+    assert st(lse=None) == fa.FA_ERR_INVALID_ARG
+    assert st(dk=264) == fa.FA_ERR_INVALID_ARG       # misaligned
+    assert st(lse=514) == fa.FA_ERR_INVALID_ARG      # misaligned lse
+    assert st(d=96) == fa.FA_ERR_UNSUPPORTED
+    assert st(Hq=3, Hkv=2) == fa.FA_ERR_UNSUPPORTED
+    assert st(scale=-1.0) == fa.FA_ERR_INVALID_ARG
+    assert st(ws=None) == fa.FA_ERR_WORKSPACE
+    assert st(B=0) == fa.FA_OK
+    assert fa.fa_bwd_workspace_size(1, 64, 8192, 128) >= 8192 * 64 * 128 * 4
+
+
+def test_fp8_and_packed_reject_before_launch(lib):
+    def st8(**kw):
+        a = dict(q=256, k=256, v=256, o=256, lse=None, B=1, Hq=2, Hkv=1, Nq=8, Nk=8, d=128, scale=0.1, dq=1.0,
+                 dk=1.0, dv=1.0, causal=1, ws=256, wsb=1 << 20)
+        a.update(kw)
+        return lib.fa_fwd_fp8(a["q"], a["k"], a["v"], a["o"], a["lse"], a["B"], a["Hq"], a["Hkv"], a["Nq"], a["Nk"],
+                              a["d"], ctypes.c_float(a["scale"]), ctypes.c_float(a["dq"]), ctypes.c_float(a["dk"]),
+                              ctypes.c_float(a["dv"]), a["causal"], a["ws"], a["wsb"], None)
+    assert st8(d=64) == fa.FA_ERR_UNSUPPORTED        # e4m3 path is d = 128 only
+    assert st8(dv=0.0) == fa.FA_ERR_INVALID_ARG
+    assert st8(dq=float("inf")) == fa.FA_ERR_INVALID_ARG
+    assert st8(ws=None) == fa.FA_ERR_WORKSPACE
+    assert st8(B=0) == fa.FA_OK
+    assert fa.fa_fwd_fp8_workspace_size(1, 8, 8192, 128) == 8 * 128 * 8192
+    assert fa.fa_fwd_fp8_workspace_size(1, 8, 8192, 64) == 0
+
+    def stp(**kw):
+        a = dict(qkv=256, o=256, lse=None, B=2, H=12, N=2048, d=64, scale=0.125, causal=1, cu=None)
+        a.update(kw)
+        return lib.fa_fwd_qkvpacked(a["qkv"], a["o"], a["lse"], a["B"], a["H"], a["N"], a["d"],
+                                    ctypes.c_float(a["scale"]), a["causal"], a["cu"], None)
+    assert stp(qkv=None) == fa.FA_ERR_INVALID_ARG
+    assert stp(o=264) == fa.FA_ERR_INVALID_ARG
+    assert stp(d=80) == fa.FA_ERR_UNSUPPORTED
+    assert stp(cu=514) == fa.FA_ERR_INVALID_ARG
+    assert stp(N=0) == fa.FA_OK
+
+
+def test_tf32_workspace_and_rejects(lib):
+    assert fa.fa_fwd_workspace_size(1, 1, 1, 128, 128, 64, fa.FA_TF32, False) >= 3 * 128 * 64 * 4
+    assert fa.fa_fwd_workspace_size(1, 1, 1, 128, 128, 128, fa.FA_TF32, False) == 0
+    assert _fwd_status(lib, dt=fa.FA_TF32, d=128) == fa.FA_ERR_UNSUPPORTED
+    assert _fwd_status(lib, dt=fa.FA_TF32, cu=512) == fa.FA_ERR_UNSUPPORTED
+    assert _fwd_status(lib, dt=fa.FA_TF32) == fa.FA_ERR_WORKSPACE
