@@ -237,9 +237,20 @@ fa_status launch_bwd(const void* q, const void* k, const void* v, const BwdParam
       CUtensorMap mq64, mdo64;
       if (!make_map(&mq64, q, D, prm.Hq, rows_q, kBwdQ) || !make_map(&mdo64, prm.dout, D, prm.Hq, rows_q, kBwdQ))
         return FA_ERR_CUDA;
+      // the fp32 dQ accumulator as a TMA reduce target: {d, Hq, rows}, box 128 x 1 x 64, no swizzle
+      CUtensorMap mdq;
+      const cuuint64_t ddq[3] = {(cuuint64_t)D, (cuuint64_t)prm.Hq, (cuuint64_t)rows_q};
+      const cuuint64_t sdq[2] = {(cuuint64_t)D * 4, (cuuint64_t)prm.Hq * D * 4};
+      const cuuint32_t bdq[3] = {(cuuint32_t)D, 1, (cuuint32_t)kBwdQ};
+      const cuuint32_t edq[3] = {1, 1, 1};
+      EncodeTiledFn enc = get_encode_fn();
+      if (!enc || enc(&mdq, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, prm.dq_acc, ddq, sdq, bdq, edq,
+                      CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                      CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+        return FA_ERR_CUDA;
       const int smem = Bwd2Cfg::kSmemBytes;
       if (set_smem(fa_bwd2_kernel, smem) != cudaSuccess) return FA_ERR_CUDA;
-      fa_bwd2_kernel<<<grid, kBwdThreads, smem, st>>>(mq64, mk, mv, mdo64, prm);
+      fa_bwd2_kernel<<<grid, kBwdThreads, smem, st>>>(mq64, mk, mv, mdo64, mdq, prm);
     } else {
       auto kern = fa_bwd_kernel<D>;
       const int smem = BwdCfg<D>::kSmemBytes;

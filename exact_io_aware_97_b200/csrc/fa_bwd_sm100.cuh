@@ -461,18 +461,21 @@ struct Bwd2Cfg {
   static constexpr int kOffQ = 2 * kKTile;                          // [slots]
   static constexpr int kOffDO = kOffQ + kBwdSlots * kQTile;         // [slots]
   static constexpr int kOffDS = kOffDO + kBwdSlots * kQTile;        // [2]
-  static constexpr int kOffVec = kOffDS + 2 * kDSTile;              // [slots][lse2, D]
+  static constexpr int kStageBytes = kBwdQ * D * 4;                 // dQ of one pair, [64 q][128 d] fp32
+  static constexpr int kOffStage = kOffDS + 2 * kDSTile;
+  static constexpr int kOffVec = kOffStage + kStageBytes;           // [slots][lse2, D]
   static constexpr int kOffBar = kOffVec + kBwdSlots * 2 * kVecBytes;
   static constexpr int kNumBars = 24;
   static constexpr int kUsed = kOffBar + kNumBars * 8 + 16;
   static constexpr int kSmemBytes = kUsed + 1024;
+  static_assert(kSmemBytes <= kBwdMaxSmem, "shared memory");
   static constexpr uint32_t kColDV = 256, kColDK = 384;
 };
 
 __global__ void __launch_bounds__(kBwdThreads, 1)
     fa_bwd2_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                    const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmDO,
-                   const BwdParams p) {
+                   const __grid_constant__ CUtensorMap tmDQ, const BwdParams p) {
   using C = Bwd2Cfg;
   constexpr int D = C::D;
   extern __shared__ uint8_t smem_raw[];
@@ -490,6 +493,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   uint8_t* sQ = smem + C::kOffQ;
   uint8_t* sDO = smem + C::kOffDO;
   uint8_t* sDS = smem + C::kOffDS;
+  float* sStage = reinterpret_cast<float*>(smem + C::kOffStage);
   float* sVec = reinterpret_cast<float*>(smem + C::kOffVec);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kOffBar);
   uint64_t* kv_full = bars + 0;
@@ -501,6 +505,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   uint64_t* dq_full = bars + 13;   // [2]
   uint64_t* buf_free = bars + 15;  // [2]
   uint64_t* acc_done = bars + 17;
+  uint64_t* stage_full = bars + 18;  // the warpgroups wrote dQ of a pair into the staging tile
+  uint64_t* stage_free = bars + 19;  // its reduction has read the staging tile
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + C::kNumBars);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -530,6 +536,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       mbar_init(buf_free + x, 8);
     }
     mbar_init(acc_done, 1);
+    mbar_init(stage_full, 8);
+    mbar_init(stage_free, 1);
     fence_barrier_init();
   }
   if (warp == 1) {
@@ -541,7 +549,25 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
-  if (warp == 0) {
+  if (warp == 2) {
+    // ============================================================ dQ reductions
+    // One TMA reduce-add per pair: the staging tile [64 queries][128 d] into the fp32
+    // accumulator rows of that pair's (query head, query tile).  Queries past Nq add zeros
+    // (their dS is 0), into rows that exist or lie beyond the tensor (then skipped).
+    if (lane == 0) {
+      for (int tp = 0; tp < T; ++tp) {
+        if (!mbar_wait(stage_full, tp & 1)) break;
+        const int h = kvh * p.G + tp / ntq;
+        const int q0 = (i_lo + tp % ntq) * kBwdQ;
+        tma_reduce_add_3d(&tmDQ, sStage, 0, h, b * p.Nq + q0);
+        bulk_commit_group();
+        bulk_wait_group_read0();
+        mbar_arrive(stage_free);
+      }
+      bulk_wait_group0();
+    }
+    __syncwarp();
+  } else if (warp == 0) {
     // ============================================================ TMA producer
     if (T > 0) {
       mbar_arrive_expect_tx_elect(kv_full, 2 * C::kKTile);
@@ -647,13 +673,14 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(buf_free + bb);
-      const int h = kvh * p.G + tp / ntq;
-      const int qb0 = (i_lo + tp % ntq) * kBwdQ + 32 * wg;
-      float* base = p.dq_acc + (((size_t)b * p.Nq + qb0) * p.Hq + h) * D + r;
-      const size_t qstride = (size_t)p.Hq * D;
+      // stage row q = 32 wg + e, column d = r (lanes write consecutive d: no bank conflicts),
+      // once the previous pair's reduction has read the tile
+      if (tp >= 1 && !warp_wait(stage_free, (tp - 1) & 1)) return false;
 #pragma unroll
-      for (int e = 0; e < 32; ++e)
-        if (qb0 + e < p.Nq) red_add_f32(base + e * qstride, __uint_as_float(a[e]));
+      for (int e = 0; e < 32; ++e) sStage[(32 * wg + e) * D + r] = __uint_as_float(a[e]);
+      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+      __syncwarp();
+      if (lane == 0) mbar_arrive(stage_full);
       return true;
     };
 
