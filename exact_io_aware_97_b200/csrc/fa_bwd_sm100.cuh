@@ -438,7 +438,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
 //   S_b = TMEM[128 b, 128 b + 64), DP_b = TMEM[128 b + 64, 128 b + 128)   (b = pair & 1)
 // dV = TMEM[256, 384), dK = TMEM[384, 512).  Per pair t (buffer b):
 //   S^T = K Q^T -> S_b, dP^T = V dO^T -> DP_b                        (tcgen05, N = 64)
-//   elementwise: P^T (bf16) over S_b[0,32), dS^T (bf16) over S_b[32,64), dS to shared memory
+//   elementwise: P^T, dS^T (bf16) of warpgroup w's 32 queries over S_b[32w, 32w+16) and
+//                S_b[32w+16, 32w+32) (the columns it read), dS to shared memory
 //   dV += P^T dO, dK += dS^T Q                                        (A from TMEM)
 //   dQ^T = K^T dS -> DP_b   (M = d on the TMEM lanes, so each warp's dQ read-out covers 32
 //                            consecutive d: coalesced fp32 reductions)
@@ -500,7 +501,6 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   uint64_t* q_full = bars + 1;     // [slots]
   uint64_t* q_empty = bars + 4;    // [slots]
   uint64_t* sdp_full = bars + 7;   // [2]
-  uint64_t* ld_done = bars + 9;    // [2]
   uint64_t* pds_ready = bars + 11; // [2]
   uint64_t* dq_full = bars + 13;   // [2]
   uint64_t* buf_free = bars + 15;  // [2]
@@ -530,7 +530,6 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     }
     for (int x = 0; x < 2; ++x) {
       mbar_init(sdp_full + x, 1);
-      mbar_init(ld_done + x, 8);
       mbar_init(pds_ready + x, 8);
       mbar_init(dq_full + x, 1);
       mbar_init(buf_free + x, 8);
@@ -635,10 +634,12 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
 #pragma unroll
           for (int kk = 0; kk < kBwdQ / 16; ++kk) {
             const uint32_t acc = (tp > 0 || kk > 0) ? 1u : 0u;
-            umma_ts_elect(tmem + C::kColDV, tmem + cS + kk * 8,
-                          smem_desc_sw128(ds + kk * 16 * 128, C::kQPanel, 1024), idAcc, acc);
-            umma_ts_elect(tmem + C::kColDK, tmem + cS + 32 + kk * 8,
-                          smem_desc_sw128(qs + kk * 16 * 128, C::kQPanel, 1024), idAcc, acc);
+            // queries 16 kk .. 16 kk + 15: warpgroup kk / 2, P^T at 32 (kk / 2) + 8 (kk % 2), dS^T 16 further
+            const uint32_t pc = cS + 32 * (kk >> 1) + 8 * (kk & 1);
+            umma_ts_elect(tmem + C::kColDV, tmem + pc, smem_desc_sw128(ds + kk * 16 * 128, C::kQPanel, 1024), idAcc,
+                          acc);
+            umma_ts_elect(tmem + C::kColDK, tmem + pc + 16, smem_desc_sw128(qs + kk * 16 * 128, C::kQPanel, 1024),
+                          idAcc, acc);
           }
           // dQ^T = K^T dS: A = K (keys x d) read d-major, B = dS (keys x queries) query-major
 #pragma unroll
@@ -739,16 +740,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
           *reinterpret_cast<uint4*>(row + (((4 * wg + u) ^ (r & 7)) << 4)) =
               make_uint4(dsk[4 * u], dsk[4 * u + 1], dsk[4 * u + 2], dsk[4 * u + 3]);
       }
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(ld_done + bb);
-      if (!warp_wait(ld_done + bb, (t >> 1) & 1)) {
-        ok = false;
-        break;
-      }
-      tc_fence_after();
-      tmem_st16(tmem + lane_off + cS + 16 * wg, pk);
-      tmem_st16(tmem + lane_off + cS + 32 + 16 * wg, dsk);
+      // P^T and dS^T of this warpgroup's 32 queries go over the 32 S columns it has just read
+      // (P^T in the first 16, dS^T in the next 16), so no other warpgroup is waited for
+      tmem_st16(tmem + lane_off + cS + 32 * wg, pk);
+      tmem_st16(tmem + lane_off + cS + 32 * wg + 16, dsk);
       tmem_wait_st();
       asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
       tc_fence_before();
