@@ -500,7 +500,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   uint64_t* kv_full = bars + 0;
   uint64_t* q_full = bars + 1;     // [slots]
   uint64_t* q_empty = bars + 4;    // [slots]
-  uint64_t* sdp_full = bars + 7;   // [2]
+  uint64_t* sdp_full = bars + 7;   // [2] S^T in TMEM
+  uint64_t* dp_full = bars + 9;    // [2] dP^T in TMEM
   uint64_t* pds_ready = bars + 11; // [2]
   uint64_t* dq_full = bars + 13;   // [2]
   uint64_t* buf_free = bars + 15;  // [2]
@@ -530,6 +531,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     }
     for (int x = 0; x < 2; ++x) {
       mbar_init(sdp_full + x, 1);
+      mbar_init(dp_full + x, 1);
       mbar_init(pds_ready + x, 8);
       mbar_init(dq_full + x, 1);
       mbar_init(buf_free + x, 8);
@@ -616,6 +618,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             umma_ss_elect(tmem + cS, smem_desc_sw128(kb + ka, 16, 1024), smem_desc_sw128(qs + kq, 16, 1024), idS,
                           kk > 0 ? 1u : 0u);
           }
+          umma_commit_elect(sdp_full + bb);  // the exponentials start while dP^T is formed
 #pragma unroll
           for (int kk = 0; kk < D / 16; ++kk) {
             const uint32_t ka = (kk >> 2) * C::kKPanel + (kk & 3) * 32;
@@ -623,7 +626,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             umma_ss_elect(tmem + cDP, smem_desc_sw128(vb + ka, 16, 1024), smem_desc_sw128(ds + kq, 16, 1024), idS,
                           kk > 0 ? 1u : 0u);
           }
-          umma_commit_elect(sdp_full + bb);
+          umma_commit_elect(dp_full + bb);
         }
         if (t >= 1) {
           const int tp = t - 1, slot = tp % kBwdSlots, bb = tp & 1;
@@ -698,9 +701,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       const float* dd = sVec + (slot * 2 + 1) * kBwdQ + 32 * wg;
       uint32_t pk[16], dsk[16];
       {
-        uint32_t sv[32], dpv[32];
+        uint32_t sv[32];
         tmem_ld32(tmem + lane_off + cS + 32 * wg, sv);
-        tmem_ld32(tmem + lane_off + cDP + 32 * wg, dpv);
         // the row vectors of this warpgroup's 32 queries (broadcast reads), while TMEM loads
         float4 lv[8], dv4[8];
 #pragma unroll
@@ -714,20 +716,35 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         if (!key_ok) lim = 32;
         else if (p.causal) lim = min(32, max(0, key - diag - qfirst));
         const uint64_t tau2 = f2(tau, tau);
+        uint64_t pp[16];
 #pragma unroll
         for (int e = 0; e < 16; ++e) {
-          const float4 L = lv[e >> 1], Dv = dv4[e >> 1];
+          const float4 L = lv[e >> 1];
           const uint64_t nl = (e & 1) ? f2(-L.z, -L.w) : f2(-L.x, -L.y);
-          const uint64_t nd = (e & 1) ? f2(-Dv.z, -Dv.w) : f2(-Dv.x, -Dv.y);
           float x0, x1;
           f2_split(f2_fma(f2(__uint_as_float(sv[2 * e]), __uint_as_float(sv[2 * e + 1])), tau2, nl), x0, x1);
           float p0 = ex2_approx(x0), p1 = ex2_approx(x1);
           if (2 * e < lim) p0 = 0.f;
           if (2 * e + 1 < lim) p1 = 0.f;
           pk[e] = pack_bf16x2(p0, p1);
+          pp[e] = f2(p0, p1);
+        }
+        // dP^T of the pair (its products were issued after S^T's)
+        if (!warp_wait(dp_full + bb, (t >> 1) & 1)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        uint32_t dpv[32];
+        tmem_ld32(tmem + lane_off + cDP + 32 * wg, dpv);
+        tmem_wait_ld();
+#pragma unroll
+        for (int e = 0; e < 16; ++e) {
+          const float4 Dv = dv4[e >> 1];
+          const uint64_t nd = (e & 1) ? f2(-Dv.z, -Dv.w) : f2(-Dv.x, -Dv.y);
           const uint64_t g2 = f2_add(f2(__uint_as_float(dpv[2 * e]), __uint_as_float(dpv[2 * e + 1])), nd);
           float g0, g1;
-          f2_split(f2_fma(f2(p0, p1), g2, f2(0.f, 0.f)), g0, g1);
+          f2_split(f2_fma(pp[e], g2, f2(0.f, 0.f)), g0, g1);
           dsk[e] = pack_bf16x2(g0, g1);
         }
       }
