@@ -19,7 +19,7 @@ FA_BF16, FA_F32, FA_TF32 = 0, 1, 2
 
 EXPORTED = ("fa_fwd", "fa_fwd_workspace_size", "fa_decode", "fa_decode_workspace_size", "fa_decode_noalloc",
             "fa_decode_paged", "fa_decode_paged_workspace_size", "fa_bwd", "fa_bwd_workspace_size", "fa_fwd_qkvpacked",
-            "fa_fwd_fp8", "fa_fwd_fp8_workspace_size",
+            "fa_fwd_fp8", "fa_fwd_fp8_workspace_size", "fa_selftest_wait_timeout",
             "fa_last_device_error", "fa_status_string", "fa_device_sm_count")
 FA_DECODE_NOALLOC_SCRATCH_BYTES = 16 << 20
 
@@ -66,6 +66,8 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
     L.fa_bwd.restype = i
     L.fa_bwd_workspace_size.argtypes = [i, i, i, i]
     L.fa_bwd_workspace_size.restype = sz
+    L.fa_selftest_wait_timeout.argtypes = [vp]
+    L.fa_selftest_wait_timeout.restype = i
     L.fa_last_device_error.argtypes = [vp]
     L.fa_last_device_error.restype = i
     L.fa_status_string.argtypes = [i]
@@ -180,6 +182,11 @@ def fa_bwd(q, k, v, o, dout, lse, dq, dk, dv, B, Hq, Hkv, Nq, Nk, d, scale, caus
 
 def fa_bwd_workspace_size(B, Hq, Nq, d) -> int:
     return int(load().fa_bwd_workspace_size(int(B), int(Hq), int(Nq), int(d)))
+
+
+def fa_selftest_wait_timeout(stream=None) -> None:
+    """Launch the self-test whose bounded wait must run out (see include/fa.h)."""
+    _check(load().fa_selftest_wait_timeout(_stream(stream)), "fa_selftest_wait_timeout")
 
 
 def fa_last_device_error(stream=None) -> int:

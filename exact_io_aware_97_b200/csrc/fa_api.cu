@@ -732,6 +732,30 @@ fa_status fa_last_device_error(void* stream) {
 }  // extern "C"
 
 // ---------------------------------------------------------------------------------------
+// Self-test of the bounded waits: one barrier that nothing arrives on.
+namespace fa {
+namespace {
+
+__global__ void selftest_wait_kernel() {
+  __shared__ uint64_t bar;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    fence_barrier_init();
+  }
+  __syncthreads();
+  // phase 0 never completes: the wait gives up after its limit, records the timeout and returns
+  if (threadIdx.x == 0) (void)mbar_wait(&bar, 0);
+}
+
+}  // namespace
+}  // namespace fa
+
+extern "C" fa_status fa_selftest_wait_timeout(void* stream) {
+  fa::selftest_wait_kernel<<<1, 32, 0, reinterpret_cast<cudaStream_t>(stream)>>>();
+  return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+}
+
+// ---------------------------------------------------------------------------------------
 // fa_decode_noalloc: fa_decode with its scratch in a static device array, for callers that
 // cannot allocate device memory (see include/fa.h).
 namespace fa {

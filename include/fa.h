@@ -223,6 +223,12 @@ FA_EXPORT size_t fa_decode_paged_workspace_size(int B, int Hq, int Hkv, int max_
  * if the stream reports an error; else FA_OK. */
 FA_EXPORT fa_status fa_last_device_error(void* stream);
 
+/* Test support for the failure detection: launches one kernel whose single wait can never be
+ * satisfied (nothing arrives on its barrier).  The wait is bounded like every wait of the
+ * library: after its time limit (4 s) it records a timeout and the kernel returns, so nothing
+ * hangs and the context stays usable; the next fa_last_device_error reports FA_ERR_TIMEOUT. */
+FA_EXPORT fa_status fa_selftest_wait_timeout(void* stream);
+
 /* Static description of a status code. */
 FA_EXPORT const char* fa_status_string(fa_status s);
 
