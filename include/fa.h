@@ -1,8 +1,8 @@
 /* Exact IO-aware attention for NVIDIA B200 (sm_100a): C ABI.
  *
- * Two operations, both computing exactly O = softmax(Q K^T * scale) V and the per-row
- * logsumexp, tile by tile with the online-softmax running max m and sum l, so the N x N
- * score and probability matrices never reach device memory:
+ * Exact attention O = softmax(Q K^T * scale) V with the per-row logsumexp, computed tile by
+ * tile with the online-softmax running max m and sum l, so the N x N score and probability
+ * matrices never reach device memory; its backward; and the decode step over a KV cache:
  *
  *   fa_fwd     the tiled forward ("FlashAttention notes", section 3 "Tiling" and section 4
  *              "Online Softmax": m_new = max(m1, m2), l_new = e^(m1-m_new) l1 + e^(m2-m_new) l2;
@@ -23,7 +23,8 @@
  *     allocates or frees device memory and never synchronises, except in
  *     fa_last_device_error.  Every launch is asynchronous on `stream` (a cudaStream_t
  *     passed as void*; NULL is the legacy default stream).
- *   - Tensors are contiguous with the head dimension d innermost.  bf16 is IEEE bfloat16.
+ *   - Tensors are contiguous with the head dimension d innermost (fa_fwd_qkvpacked reads
+ *     its three slices with a row stride of 3 H d).  bf16 is IEEE bfloat16.
  *   - Arguments are validated on the host before anything is launched; a rejected call
  *     returns FA_ERR_INVALID_ARG or FA_ERR_UNSUPPORTED and touches no memory.
  *   - A failed launch returns FA_ERR_CUDA.  A device-side wait that exceeded its time
