@@ -53,3 +53,18 @@ def test_aggregate_rate_counts_all_ranks():
 
 def test_single_process_max_is_identity():
     assert bench.max_over_ranks(3.25) == 3.25
+
+
+def test_json_line_has_no_nan():
+    """Phases left out with --only report null (NaN is not JSON)."""
+    import json
+    line = {"value": float("nan"), "nested": {"x": [1.0, float("nan")], "y": "s"}, "z": 2}
+    out = json.dumps(bench._nan_to_null(line), allow_nan=False)
+    assert json.loads(out) == {"value": None, "nested": {"x": [1.0, None], "y": "s"}, "z": 2}
+
+
+def test_paged_workload_bytes_follow_lengths():
+    w = bench.PAGED
+    lens = bench.paged_lengths(w["seed"])
+    assert len(lens) == w["B"] and lens.min() >= w["len_lo"] and lens.max() <= w["len_hi"]
+    assert bench.paged_kv_bytes(lens) == 2.0 * lens.sum() * w["Hkv"] * w["d"] * 2
