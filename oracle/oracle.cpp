@@ -76,7 +76,11 @@ RowView view_row(const Problem& P, int b, int h, int64_t i) {
     q0 = P.cu[b];
     k0 = P.cu[b];
     nq = P.cu[b + 1] - P.cu[b];
+#ifdef ORACLE_PLANT_VARLEN_SHORT_KEYS
+    nk = nq > 0 ? nq - 1 : 0;
+#else
     nk = nq;
+#endif
   } else {
     q0 = (int64_t)b * P.Nq;
     k0 = (int64_t)b * P.Nk;

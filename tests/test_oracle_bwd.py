@@ -7,10 +7,13 @@ come from the oracle's backward itself:
 * torch.autograd (fp64, CPU) on the plain formula softmax(scale q k^T + mask) v, with GQA
   written as repeating each key/value head over its group;
 * invariants: sum_j dV_j = sum_i dO_i over a group (rows of P sum to 1); dQ does not change
-  when one vector is added to every key (rows of dS sum to 0); dQ = 0 when all keys are equal.
+  when one vector is added to every key (rows of dS sum to 0); dQ = 0 when all keys are equal;
+* packed variable-length sequences give each sequence's own gradients (no attention, hence
+  no gradient, crosses a sequence boundary).
 
 Planted mistakes (a dropped D term, dK built from P instead of dS, dQ without the scale, the
-GQA and causal mistakes of the forward pins) must each fail at least one pin.
+GQA and causal mistakes of the forward pins, a packed sequence that loses its last key) must
+each fail at least one pin.
 """
 import numpy as np
 import pytest
@@ -98,7 +101,30 @@ def pin_invariants(orc):
     return ok
 
 
-PINS = [pin_finite_differences, pin_autograd, pin_invariants]
+def pin_varlen_equals_independent(orc):
+    """Packed sequences (an empty one included) give the gradients of each sequence run on
+    its own: attention never crosses a sequence boundary, so neither does a gradient."""
+    lens = [4, 9, 1, 0, 6]
+    cu = si.cu_seqlens(lens)
+    T, Hq, Hkv, d = int(cu[-1]), 4, 2, 4
+    q = _rand((T, Hq, d), 8401, si.Q)
+    k = _rand((T, Hkv, d), 8401, si.K)
+    v = _rand((T, Hkv, d), 8401, si.V)
+    do = _rand((T, Hq, d), 8401, 9)
+    ok = True
+    for causal in (False, True):
+        dq, dk, dv = orc.attention_bwd(q, k, v, do, 0.5, causal=causal, cu_seqlens=cu)
+        for b in range(len(lens)):
+            s = slice(int(cu[b]), int(cu[b + 1]))
+            if lens[b] == 0:
+                continue
+            gq, gk, gv = orc.attention_bwd(q[s][None], k[s][None], v[s][None], do[s][None], 0.5, causal=causal)
+            ok &= np.allclose(dq[s], gq[0], atol=1e-14) and np.allclose(dk[s], gk[0], atol=1e-14)
+            ok &= np.allclose(dv[s], gv[0], atol=1e-14)
+    return bool(ok)
+
+
+PINS = [pin_finite_differences, pin_autograd, pin_invariants, pin_varlen_equals_independent]
 
 
 @pytest.fixture(scope="module")
@@ -113,7 +139,7 @@ def test_bwd_pin(orc, pin):
 
 @pytest.mark.parametrize("plant", ["ORACLE_PLANT_BWD_NO_D", "ORACLE_PLANT_BWD_DK_FROM_P",
                                    "ORACLE_PLANT_BWD_DQ_NO_SCALE", "ORACLE_PLANT_GQA_MODULO",
-                                   "ORACLE_PLANT_CAUSAL_OFF_BY_ONE"])
+                                   "ORACLE_PLANT_CAUSAL_OFF_BY_ONE", "ORACLE_PLANT_VARLEN_SHORT_KEYS"])
 def test_bwd_pins_catch_planted_mistake(plant):
     broken = oracle_mod.build_planted(plant)
     assert not all(pin(broken) for pin in PINS)

@@ -389,7 +389,8 @@ def test_pin(orc, pin):
 
 
 PLANTS = ["ORACLE_PLANT_NO_SCALE", "ORACLE_PLANT_SIGN", "ORACLE_PLANT_QV_SWAP",
-          "ORACLE_PLANT_LSE_NO_MAX", "ORACLE_PLANT_CAUSAL_OFF_BY_ONE", "ORACLE_PLANT_GQA_MODULO"]
+          "ORACLE_PLANT_LSE_NO_MAX", "ORACLE_PLANT_CAUSAL_OFF_BY_ONE", "ORACLE_PLANT_GQA_MODULO",
+          "ORACLE_PLANT_VARLEN_SHORT_KEYS"]
 
 
 @pytest.mark.parametrize("plant", PLANTS)
