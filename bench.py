@@ -46,6 +46,7 @@ FWD = si.WORKLOADS["gqa_causal_8k"]
 DEC = si.WORKLOADS["decode_split_kv"]
 PAGED = si.WORKLOADS["decode_paged_ragged"]
 MHA2K = si.WORKLOADS["mha_causal_2k"]
+VARLEN = si.WORKLOADS["varlen_gqa_causal"]
 DOUT_ID = 9  # stream id of the backward's upstream gradient
 
 
@@ -69,6 +70,15 @@ def paged_lengths(seed: int, w=PAGED) -> np.ndarray:
 
 def paged_kv_bytes(lengths, w=PAGED) -> float:
     return 2.0 * float(np.sum(lengths)) * w["Hkv"] * w["d"] * 2
+
+
+def varlen_lengths(seed: int, w=VARLEN) -> np.ndarray:
+    return si.varlen_lengths(seed, w["nseq"], w["len_lo"], w["len_hi"])
+
+
+def varlen_flops(lengths, w=VARLEN) -> float:
+    """Forward FLOPs of packed causal sequences: sum over sequences of 4 Hq L^2 d, halved."""
+    return float(sum(4.0 * w["Hq"] * float(L) * float(L) * w["d"] for L in lengths)) / 2.0
 
 
 def dec_flops(w=DEC) -> float:
@@ -245,6 +255,7 @@ def run_device(args):
     do_bwd = args.only in ("all", "bwd")
     do_fp8 = args.only in ("all", "fp8")
     do_tf32 = args.only in ("all", "tf32")
+    do_bwdv = args.only == "bwd_varlen"  # on request only: its inputs take about a minute to draw
     if do_bwd:
         h_do_f = torch.from_numpy(inputs("fwd", seed, DOUT_ID, (B, N, Hq, d))).to(torch.bfloat16)
         b_do = h_do_f.to(dev)
@@ -307,6 +318,27 @@ def run_device(args):
         t_ws_bytes = fa.fa_fwd_workspace_size(tB, tH, tH, tN, tN, td, fa.FA_TF32, False)
         t_ws = torch.empty(t_ws_bytes, dtype=torch.uint8, device=dev)
 
+    if do_bwdv:
+        vseed = replica_seed(VARLEN["seed"], rank)
+        v_len = varlen_lengths(vseed)
+        v_cu_np = si.cu_seqlens(v_len)
+        vT, vB = int(v_cu_np[-1]), len(v_len)
+        vHq, vHkv, vd = VARLEN["Hq"], VARLEN["Hkv"], VARLEN["d"]
+        v_q, v_k, v_v, v_do = (torch.from_numpy(inputs("varlen", vseed, tid, (vT, hh, vd))).to(torch.bfloat16).to(dev)
+                               for tid, hh in ((si.Q, vHq), (si.K, vHkv), (si.V, vHkv), (DOUT_ID, vHq)))
+        v_cu = torch.from_numpy(v_cu_np).to(dev)
+        v_o = torch.empty_like(v_q)
+        v_lse = torch.empty((vHq, vT), dtype=torch.float32, device=dev)
+        vscale = 1.0 / math.sqrt(vd)
+        fa.fa_fwd(v_q, v_k, v_v, v_o, v_lse, vB, vHq, vHkv, vT, vT, vd, vscale, 1, v_cu, fa.FA_BF16, None, 0, st)
+        v_dq, v_dk, v_dv = torch.empty_like(v_q), torch.empty_like(v_k), torch.empty_like(v_v)
+        v_ws_bytes = fa.fa_bwd_varlen_workspace_size(vB, vHq, vT, vd)
+        v_ws = torch.empty(v_ws_bytes, dtype=torch.uint8, device=dev)
+
+    def call_bwdv():
+        fa.fa_bwd_varlen(v_q, v_k, v_v, v_o, v_do, v_lse, v_dq, v_dk, v_dv, vB, vHq, vHkv, vT, vd, vscale, 1, v_cu,
+                         v_ws, v_ws_bytes, st)
+
     def call_tf32():
         fa.fa_fwd(tq, tk, tv, t_o, t_lse, tB, tH, tH, tN, tN, td, 1.0 / math.sqrt(td), 1, None, fa.FA_TF32, t_ws,
                   t_ws_bytes, st)
@@ -358,6 +390,7 @@ def run_device(args):
     bwd_ms = timed_launches(call_bwd, args.steps, args.warmup) if do_bwd else [float("nan")]
     fp8_ms = timed_launches(call_fp8, args.steps, args.warmup) if do_fp8 else [float("nan")]
     tf32_ms = timed_launches(call_tf32, args.steps, args.warmup) if do_tf32 else [float("nan")]
+    bwdv_ms = timed_launches(call_bwdv, args.steps, args.warmup) if do_bwdv else [float("nan")]
     if fa.fa_last_device_error(st) != fa.FA_OK:
         raise RuntimeError("device-side timeout recorded during the benchmark")
 
@@ -404,6 +437,7 @@ def run_device(args):
     bwd_mean = max_over_ranks(sum(bwd_ms) / len(bwd_ms), dev)
     fp8_mean = max_over_ranks(sum(fp8_ms) / len(fp8_ms), dev)
     tf32_mean = max_over_ranks(sum(tf32_ms) / len(tf32_ms), dev)
+    bwdv_mean = max_over_ranks(sum(bwdv_ms) / len(bwdv_ms), dev)
     fwd_e2e_ms = max_over_ranks(fwd_e2e_ms, dev)
     dec_e2e_ms = max_over_ranks(dec_e2e_ms, dev)
     if world > 1:
@@ -513,11 +547,27 @@ def run_device(args):
         "e2e": {"value": round(world * F / (fwd_e2e_ms * 1e-3) / 1e12, 2), "unit": "TFLOP/s",
                 "h2d_bytes_per_step": h2d_fwd, "d2h_bytes_per_step": d2h_fwd},
         "cpu_baseline": cpu,
-        "gpu_launches": args.steps * (int(do_fwd) * 1 + int(do_dec) * 2 + int(do_paged) * 1 + int(do_bwd) * 3 + int(do_fp8) * 2 + int(do_tf32) * 4)
+        "gpu_launches": args.steps * (int(do_fwd) * 1 + int(do_dec) * 2 + int(do_paged) * 1 + int(do_bwd) * 3 + int(do_fp8) * 2 + int(do_tf32) * 4
+                                     + int(do_bwdv) * 4)
         + (0 if args.no_e2e else e2e_steps * (int(do_fwd) * 1 + int(do_dec) * 2)),
         "clocks": clocks.summary(),
         "impl": "b200",
     }
+    if do_bwdv:
+        vF = 2.5 * varlen_flops(v_len)
+        v_tflops = vF / (bwdv_mean * 1e-3) / 1e12
+        v_peak = peaks["bf16"] if (args.steps * bwdv_mean) < 1000.0 else peaks["bf16_sustained"]
+        line["backward_varlen"] = {
+            "value": round(aggregate_rate(vF, world, bwdv_mean) / 1e12, 2), "unit": "TFLOP/s",
+            "ms": round(bwdv_mean, 4),
+            "workload": "varlen_gqa_causal backward: 16 packed sequences, lengths U[256, 8192] (seed 1004), "
+                        "Hq=32, Hkv=8, d=128, causal",
+            "flops_convention": "2.5 x the sequences' causal forward FLOPs",
+            "roofline": {"bound": "tensor", "achieved": round(v_tflops, 2), "peak": v_peak, "unit": "TFLOP/s",
+                         "frac": round(v_tflops / v_peak, 4), "peak_kind": f"measured ({peaks['source']})",
+                         "kernels": "fa_bwd_tiles_kernel + fa_bwd_pre_kernel<128> + fa_bwd2_kernel + "
+                                    "fa_bwd_dq_kernel<128>",
+                         "algorithmic_flops_per_launch": vF}}
     print(json.dumps(_nan_to_null(line)), flush=True)
 
 
@@ -645,7 +695,7 @@ def main():
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--no-cpu", action="store_true", help="skip the CPU oracle baseline")
     ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer end-to-end phases")
-    ap.add_argument("--only", default="all", choices=["all", "fwd", "dec", "paged", "bwd", "fp8", "tf32"],
+    ap.add_argument("--only", default="all", choices=["all", "fwd", "dec", "paged", "bwd", "fp8", "tf32", "bwd_varlen"],
                     help="profiling: run one kernel family")
     args = ap.parse_args()
     if args.warmup < 3:

@@ -18,7 +18,8 @@ FA_OK, FA_ERR_INVALID_ARG, FA_ERR_UNSUPPORTED, FA_ERR_WORKSPACE, FA_ERR_CUDA, FA
 FA_BF16, FA_F32, FA_TF32 = 0, 1, 2
 
 EXPORTED = ("fa_fwd", "fa_fwd_workspace_size", "fa_decode", "fa_decode_workspace_size", "fa_decode_noalloc",
-            "fa_decode_paged", "fa_decode_paged_workspace_size", "fa_bwd", "fa_bwd_workspace_size", "fa_fwd_qkvpacked",
+            "fa_decode_paged", "fa_decode_paged_workspace_size", "fa_bwd", "fa_bwd_workspace_size", "fa_bwd_varlen",
+            "fa_bwd_varlen_workspace_size", "fa_fwd_qkvpacked",
             "fa_fwd_fp8", "fa_fwd_fp8_workspace_size", "fa_selftest_wait_timeout",
             "fa_last_device_error", "fa_status_string", "fa_device_sm_count")
 FA_DECODE_NOALLOC_SCRATCH_BYTES = 16 << 20
@@ -66,6 +67,10 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
     L.fa_bwd.restype = i
     L.fa_bwd_workspace_size.argtypes = [i, i, i, i]
     L.fa_bwd_workspace_size.restype = sz
+    L.fa_bwd_varlen.argtypes = [vp] * 9 + [i] * 5 + [f, i, vp, vp, sz, vp]
+    L.fa_bwd_varlen.restype = i
+    L.fa_bwd_varlen_workspace_size.argtypes = [i, i, i, i]
+    L.fa_bwd_varlen_workspace_size.restype = sz
     L.fa_selftest_wait_timeout.argtypes = [vp]
     L.fa_selftest_wait_timeout.restype = i
     L.fa_last_device_error.argtypes = [vp]
@@ -184,6 +189,19 @@ def fa_bwd_workspace_size(B, Hq, Nq, d) -> int:
     return int(load().fa_bwd_workspace_size(int(B), int(Hq), int(Nq), int(d)))
 
 
+def fa_bwd_varlen(q, k, v, o, dout, lse, dq, dk, dv, B, Hq, Hkv, total, d, scale, causal, cu_seqlens, workspace,
+                  workspace_bytes, stream=None) -> None:
+    st = load().fa_bwd_varlen(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(dout), _ptr(lse), _ptr(dq), _ptr(dk),
+                              _ptr(dv), int(B), int(Hq), int(Hkv), int(total), int(d), float(scale),
+                              int(bool(causal)), _ptr(cu_seqlens), _ptr(workspace), int(workspace_bytes),
+                              _stream(stream))
+    _check(st, "fa_bwd_varlen")
+
+
+def fa_bwd_varlen_workspace_size(B, Hq, total, d) -> int:
+    return int(load().fa_bwd_varlen_workspace_size(int(B), int(Hq), int(total), int(d)))
+
+
 def fa_selftest_wait_timeout(stream=None) -> None:
     """Launch the self-test whose bounded wait must run out (see include/fa.h)."""
     _check(load().fa_selftest_wait_timeout(_stream(stream)), "fa_selftest_wait_timeout")
@@ -286,6 +304,24 @@ def backward(q, k, v, o, lse, dout, causal=False, scale=None, workspace=None, st
     if workspace is None:
         workspace = torch.empty(max(ws_bytes, 1), dtype=torch.uint8, device=q.device)
     fa_bwd(q, k, v, o, dout, lse, dq, dk, dv, B, Hq, Hkv, Nq, Nk, d, scale, causal, workspace, ws_bytes, stream)
+    return dq, dk, dv
+
+
+def backward_varlen(q, k, v, o, lse, dout, cu_seqlens, causal=False, scale=None, workspace=None, stream=None):
+    """dq, dk, dv for packed sequences: q, o, dout [total,Hq,d], k/v [total,Hkv,d], lse [Hq,total]
+    from the varlen forward, cu_seqlens int32 [B+1] on the device."""
+    import torch
+    total, Hq, d = q.shape
+    Hkv = k.shape[1]
+    B = cu_seqlens.numel() - 1
+    if scale is None:
+        scale = d ** -0.5
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    ws_bytes = fa_bwd_varlen_workspace_size(B, Hq, total, d)
+    if workspace is None:
+        workspace = torch.empty(max(ws_bytes, 1), dtype=torch.uint8, device=q.device)
+    fa_bwd_varlen(q, k, v, o, dout, lse, dq, dk, dv, B, Hq, Hkv, total, d, scale, causal, cu_seqlens, workspace,
+                  ws_bytes, stream)
     return dq, dk, dv
 
 

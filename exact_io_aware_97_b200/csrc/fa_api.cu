@@ -217,21 +217,28 @@ fa_status launch_decode_paged(const void* kp, const void* vp, const DecParams& p
   return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
 
+// Fixed length (prm.cu null) or packed varlen rows (prm.cu, prm.total, prm.ntiles set).
 template <int D>
 fa_status launch_bwd(const void* q, const void* k, const void* v, const BwdParams& prm, cudaStream_t st) {
   CUtensorMap mq, mk, mv, mdo;
-  const int64_t rows_q = (int64_t)prm.B * prm.Nq, rows_k = (int64_t)prm.B * prm.Nk;
+  const bool varlen = prm.cu != nullptr;
+  const int64_t rows_q = varlen ? (int64_t)prm.total : (int64_t)prm.B * prm.Nq;
+  const int64_t rows_k = varlen ? (int64_t)prm.total : (int64_t)prm.B * prm.Nk;
   if (!make_map(&mq, q, D, prm.Hq, rows_q, kBwdTile) || !make_map(&mdo, prm.dout, D, prm.Hq, rows_q, kBwdTile) ||
       !make_map(&mk, k, D, prm.Hkv, rows_k, kBwdTile) || !make_map(&mv, v, D, prm.Hkv, rows_k, kBwdTile))
     return FA_ERR_CUDA;
   const int sms = sm_count_cached();
   if (sms <= 0) return FA_ERR_CUDA;
-  const long long pre_rows = (long long)prm.B * prm.Hq * prm.NqPad;
+  if (varlen) fa_bwd_tiles_kernel<<<1, kTilesThreads, 0, st>>>(prm);
+  const long long pre_rows =
+      varlen ? (long long)prm.Hq * prm.ntiles * kBwdTile : (long long)prm.B * prm.Hq * prm.NqPad;
   const int pre_blocks = (int)std::min<long long>((pre_rows + 7) / 8, (long long)sms * 16);
   if (pre_blocks > 0) fa_bwd_pre_kernel<D><<<pre_blocks, 256, 0, st>>>(prm);
   if (cudaGetLastError() != cudaSuccess) return FA_ERR_CUDA;
-  if (prm.Nk > 0) {
-    dim3 grid((prm.Nk + kBwdTile - 1) / kBwdTile, prm.Hkv, prm.B);
+  if (rows_k > 0 && (varlen || prm.Nk > 0)) {
+    // varlen: one CTA index per tile of any sequence (bounded by ntiles; the kernels find
+    // the sequence and leave indices past the last tile idle)
+    const dim3 grid = varlen ? dim3(prm.ntiles, prm.Hkv, 1) : dim3((prm.Nk + kBwdTile - 1) / kBwdTile, prm.Hkv, prm.B);
     if (D == 128) {
       // pairs of 64 queries, two in flight: Q and dO maps with 64-row boxes
       CUtensorMap mq64, mdo64;
@@ -259,7 +266,7 @@ fa_status launch_bwd(const void* q, const void* k, const void* v, const BwdParam
     }
     if (cudaGetLastError() != cudaSuccess) return FA_ERR_CUDA;
   }
-  const size_t n4 = (size_t)prm.B * prm.Nq * prm.Hq * D / 4;
+  const size_t n4 = (size_t)rows_q * prm.Hq * D / 4;
   if (n4 > 0) fa_bwd_dq_kernel<D><<<(int)std::min<size_t>((n4 + 255) / 256, (size_t)sms * 8), 256, 0, st>>>(prm);
   return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
@@ -711,6 +718,66 @@ fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, con
       return FA_ERR_CUDA;
     return FA_OK;
   }
+  return d == 64 ? launch_bwd<64>(q, k, v, prm, st) : launch_bwd<128>(q, k, v, prm, st);
+}
+
+// Varlen backward: the tile bound and the workspace carve (tile prefix sums, two row vectors,
+// the fp32 dq accumulator).
+static int64_t bwd_varlen_ntiles(int B, int total) { return std::max<int64_t>(1, ((int64_t)total + 127 * (int64_t)B) / kBwdTile); }
+
+size_t fa_bwd_varlen_workspace_size(int B, int Hq, int total, int d) {
+  if (B <= 0 || Hq <= 0 || total <= 0 || d <= 0) return 0;
+  const size_t vec = (size_t)Hq * bwd_varlen_ntiles(B, total) * kBwdTile * 4;
+  return align_up((size_t)(B + 1) * 4, 256) + 2 * align_up(vec, 256) + align_up((size_t)total * Hq * d * 4, 256);
+}
+
+fa_status fa_bwd_varlen(const void* q, const void* k, const void* v, const void* o, const void* dout, const float* lse,
+                        void* dq, void* dk, void* dv, int B, int Hq, int Hkv, int total, int d, float scale,
+                        int causal, const int32_t* cu_seqlens, void* workspace, size_t workspace_bytes,
+                        void* stream) {
+  if (!q || !k || !v || !o || !dout || !lse || !dq || !dk || !dv || !cu_seqlens) return FA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(dout) || !aligned16(dq) ||
+      !aligned16(dk) || !aligned16(dv) || (reinterpret_cast<uintptr_t>(lse) & 3u) != 0 ||
+      (reinterpret_cast<uintptr_t>(cu_seqlens) & 3u) != 0)
+    return FA_ERR_INVALID_ARG;
+  if (B < 0 || Hq <= 0 || Hkv <= 0 || total < 0) return FA_ERR_INVALID_ARG;
+  if (!(scale > 0.f) || !std::isfinite(scale)) return FA_ERR_INVALID_ARG;
+  if (Hq % Hkv != 0) return FA_ERR_UNSUPPORTED;
+  if (d != 64 && d != 128) return FA_ERR_UNSUPPORTED;
+  if (Hkv > 65535) return FA_ERR_UNSUPPORTED;
+  if (B == 0 || total == 0) return FA_OK;
+  const int64_t ntiles = bwd_varlen_ntiles(B, total);
+  if (ntiles * kBwdTile >= (int64_t(1) << 31)) return FA_ERR_UNSUPPORTED;
+  const size_t need = fa_bwd_varlen_workspace_size(B, Hq, total, d);
+  if (!workspace || workspace_bytes < need || !aligned16(workspace)) return FA_ERR_WORKSPACE;
+  const size_t vec = align_up((size_t)Hq * ntiles * kBwdTile * 4, 256);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  BwdParams prm{};
+  prm.tiles = reinterpret_cast<int32_t*>(ws);
+  ws += align_up((size_t)(B + 1) * 4, 256);
+  prm.lse2 = reinterpret_cast<float*>(ws);
+  prm.dvec = reinterpret_cast<float*>(ws + vec);
+  prm.dq_acc = reinterpret_cast<float*>(ws + 2 * vec);
+  prm.o = static_cast<const __nv_bfloat16*>(o);
+  prm.dout = static_cast<const __nv_bfloat16*>(dout);
+  prm.lse = lse;
+  prm.dq = static_cast<__nv_bfloat16*>(dq);
+  prm.dk = static_cast<__nv_bfloat16*>(dk);
+  prm.dv = static_cast<__nv_bfloat16*>(dv);
+  prm.B = B;
+  prm.Hq = Hq;
+  prm.Hkv = Hkv;
+  prm.G = Hq / Hkv;
+  prm.Nq = total;
+  prm.Nk = total;
+  prm.NqPad = 0;
+  prm.causal = causal ? 1 : 0;
+  prm.scale = scale;
+  prm.tau = (float)((double)scale * 1.4426950408889634074);
+  prm.cu = cu_seqlens;
+  prm.ntiles = (int)ntiles;
+  prm.total = total;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   return d == 64 ? launch_bwd<64>(q, k, v, prm, st) : launch_bwd<128>(q, k, v, prm, st);
 }
 

@@ -55,11 +55,21 @@ struct BwdParams {
   int causal;
   float tau;    // scale * log2(e)
   float scale;
+  // packed variable-length sequences (null cu: fixed length).  Sequence b holds rows
+  // [cu[b], cu[b+1]) of q, k, v, o, dO and their gradients; lse is [Hq, total].  Key tiles
+  // of all sequences are numbered in order: tiles[b] = 128-row tiles of sequences before b.
+  // The row vectors hold, per head, ntiles * 128 entries; sequence b's queries start at
+  // entry tiles[b] * 128, padded to whole tiles.
+  const int32_t* cu;  // [B + 1]
+  int32_t* tiles;     // [B + 1], written by fa_bwd_tiles_kernel
+  int ntiles;         // bound on tiles[B]: the CTA index space and the vector stride / 128
+  int total;          // packed rows
 };
 
 constexpr int kBwdThreads = 384;
 constexpr int kBwdTile = 128;            // keys per CTA tile and queries per pair
 constexpr unsigned int kErrSmem = 4u;    // the kernel's shared-memory carve did not fit
+constexpr unsigned int kErrBadSeqlens = 8u;  // cu_seqlens not non-decreasing within [0, total]
 constexpr int kBwdMaxSmem = 232448;      // sm_100 per-block limit
 
 template <int D>
@@ -81,20 +91,143 @@ struct BwdCfg {
   static constexpr uint32_t kColS = 0, kColDP = 128, kColDV = 256, kColDK = 256 + D;
 };
 
+// Where one CTA's 128-key tile lies.  Fixed length: sequence z, tile x.  Varlen: x numbers
+// the tiles of all sequences in order; the sequence is found by bisection over the tile
+// prefix sums, and an index at or past the last tile has no work.
+struct BwdSeq {
+  int tile;        // the tile within its sequence
+  int nq, nk;      // query and key rows of the sequence
+  int rowq, rowk;  // its first row in the q-side (q, o, dO, dQ) and k-side (k, v, dK, dV) rows
+  long long vec0;  // row-vector entry of (head 0, query 0); head h adds h * vech
+  long long vech;
+};
+
+// Largest b in [0, B] with tiles[b] <= x (B: x is at or past the last tile).
+__device__ __forceinline__ int bwd_find_seq(const BwdParams& p, int x) {
+  int lo = 0, hi = p.B;
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (__ldg(p.tiles + mid) <= x) lo = mid;
+    else hi = mid - 1;
+  }
+  return lo;
+}
+
+__device__ __forceinline__ bool bwd_locate(const BwdParams& p, int x, int z, BwdSeq& s) {
+  if (p.cu == nullptr) {
+    s.tile = x;
+    s.nq = p.Nq;
+    s.nk = p.Nk;
+    s.rowq = z * p.Nq;
+    s.rowk = z * p.Nk;
+    s.vech = p.NqPad;
+    s.vec0 = (long long)z * p.Hq * p.NqPad;
+    return true;
+  }
+  const int b = bwd_find_seq(p, x);
+  if (b >= p.B) return false;
+  const int t0 = __ldg(p.tiles + b);
+  const int c0 = __ldg(p.cu + b);
+  s.tile = x - t0;
+  s.nq = s.nk = __ldg(p.cu + b + 1) - c0;
+  s.rowq = s.rowk = c0;
+  s.vech = (long long)p.ntiles * kBwdTile;
+  s.vec0 = (long long)t0 * kBwdTile;
+  return true;
+}
+
+// ------------------------------------------------------------------ varlen: tile prefix sums
+// One block: tiles[b] = sum over sequences before b of ceil(len / 128).  cu must start at or
+// above 0, never decrease and end at or below total; otherwise every entry is 0 (no CTA of
+// the main kernel has work) and kErrBadSeqlens is recorded.
+constexpr int kTilesThreads = 1024;
+__global__ void __launch_bounds__(kTilesThreads) fa_bwd_tiles_kernel(const BwdParams p) {
+  __shared__ int warp_sum[kTilesThreads / 32];
+  const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
+  const int per = (p.B + kTilesThreads - 1) / kTilesThreads;
+  const int b0 = min(p.B, t * per), b1 = min(p.B, b0 + per);
+  int sum = 0, bad = 0;
+  for (int b = b0; b < b1; ++b) {
+    const int c0 = __ldg(p.cu + b), c1 = __ldg(p.cu + b + 1);
+    bad |= (c1 < c0) | (b == 0 && c0 < 0) | (b == p.B - 1 && c1 > p.total);
+    sum += (max(c1 - c0, 0) + kBwdTile - 1) / kBwdTile;
+  }
+  // exclusive prefix of the per-thread sums: within the warp, then over the warp totals
+  int incl = sum;
+#pragma unroll
+  for (int off = 1; off < 32; off <<= 1) {
+    const int y = __shfl_up_sync(0xffffffffu, incl, off);
+    if (lane >= off) incl += y;
+  }
+  if (lane == 31) warp_sum[warp] = incl;
+  bad = __syncthreads_or(bad);
+  if (warp == 0) {
+    int w = warp_sum[lane];
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, w, off);
+      if (lane >= off) w += y;
+    }
+    warp_sum[lane] = w;  // inclusive over warps
+  }
+  __syncthreads();
+  int run = incl - sum + (warp > 0 ? warp_sum[warp - 1] : 0);
+  const int grand = warp_sum[kTilesThreads / 32 - 1];
+  bad |= grand > p.ntiles;
+  if (bad) {
+    for (int b = t; b <= p.B; b += kTilesThreads) p.tiles[b] = 0;
+    if (t == 0) atomicOr(&g_error_word, kErrBadSeqlens);
+    return;
+  }
+  for (int b = b0; b < b1; ++b) {
+    p.tiles[b] = run;
+    run += (__ldg(p.cu + b + 1) - __ldg(p.cu + b) + kBwdTile - 1) / kBwdTile;
+  }
+  if (t == 0) p.tiles[p.B] = grand;
+}
+
 // ------------------------------------------------------------------ pre: D and lse2, zero dQ
 template <int D>
 __global__ void __launch_bounds__(256) fa_bwd_pre_kernel(const BwdParams p) {
   const int warps = blockDim.x >> 5;
   const int lane = threadIdx.x & 31;
-  const long long rows = (long long)p.B * p.Hq * p.NqPad;
   constexpr int E = D / 32;  // elements per lane
+  const bool varlen = p.cu != nullptr;
+  const long long per_head = (long long)p.ntiles * kBwdTile;  // varlen vector entries per head
+  const long long rows = varlen ? per_head * p.Hq : (long long)p.B * p.Hq * p.NqPad;
+  if (varlen) {
+    // the accumulator as one flat range (rows outside every sequence included)
+    const size_t n4 = (size_t)p.total * p.Hq * D / 4;
+    for (size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x; i < n4; i += (size_t)gridDim.x * blockDim.x)
+      reinterpret_cast<float4*>(p.dq_acc)[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+  }
   for (long long w = (long long)blockIdx.x * warps + (threadIdx.x >> 5); w < rows; w += (long long)gridDim.x * warps) {
-    const int q = (int)(w % p.NqPad);
-    const long long bh = w / p.NqPad;
-    const int h = (int)(bh % p.Hq), b = (int)(bh / p.Hq);
+    // vector entry w -> row of o / dO (units of D; -1: padding) and lse index
+    long long row = -1, li = 0;
+    if (!varlen) {
+      const int q = (int)(w % p.NqPad);
+      const long long bh = w / p.NqPad;
+      const int h = (int)(bh % p.Hq);
+      const int b = (int)(bh / p.Hq);
+      if (q < p.Nq) {
+        row = ((long long)b * p.Nq + q) * p.Hq + h;
+        li = ((long long)b * p.Hq + h) * p.Nq + q;
+      }
+    } else {
+      const int h = (int)(w / per_head);
+      const int pos = (int)(w - h * per_head);
+      const int b = bwd_find_seq(p, pos / kBwdTile);
+      if (b < p.B) {
+        const int c0 = __ldg(p.cu + b);
+        const int q = pos - __ldg(p.tiles + b) * kBwdTile;
+        if (q < __ldg(p.cu + b + 1) - c0) {
+          row = ((long long)c0 + q) * p.Hq + h;
+          li = (long long)h * p.total + c0 + q;
+        }
+      }
+    }
     float dsum = 0.f, l2 = INFINITY;
-    if (q < p.Nq) {
-      const size_t row = ((size_t)b * p.Nq + q) * p.Hq + h;
+    if (row >= 0) {
       const __nv_bfloat16* orow = p.o + row * D + lane * E;
       const __nv_bfloat16* drow = p.dout + row * D + lane * E;
 #pragma unroll
@@ -103,10 +236,12 @@ __global__ void __launch_bounds__(256) fa_bwd_pre_kernel(const BwdParams p) {
         const float2 g = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(drow + e));
         dsum = fmaf(a.x, g.x, fmaf(a.y, g.y, dsum));
       }
-      float* acc = p.dq_acc + row * D + lane * E;
+      if (!varlen) {
+        float* acc = p.dq_acc + row * D + lane * E;
 #pragma unroll
-      for (int e = 0; e < E; ++e) acc[e] = 0.f;
-      const float l = p.lse[((size_t)b * p.Hq + h) * p.Nq + q];
+        for (int e = 0; e < E; ++e) acc[e] = 0.f;
+      }
+      const float l = p.lse[li];
       l2 = (l == -INFINITY) ? INFINITY : l * 1.4426950408889634f;
     }
 #pragma unroll
@@ -121,7 +256,8 @@ __global__ void __launch_bounds__(256) fa_bwd_pre_kernel(const BwdParams p) {
 // ------------------------------------------------------------------ post: dQ to bf16
 template <int D>
 __global__ void __launch_bounds__(256) fa_bwd_dq_kernel(const BwdParams p) {
-  const size_t n4 = (size_t)p.B * p.Nq * p.Hq * D / 4;
+  const size_t rows = p.cu != nullptr ? (size_t)p.total : (size_t)p.B * p.Nq;
+  const size_t n4 = rows * p.Hq * D / 4;
   const size_t stride = (size_t)gridDim.x * blockDim.x;
   for (size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x; i < n4; i += stride) {
     const float4 x = reinterpret_cast<const float4*>(p.dq_acc)[i];
@@ -168,10 +304,13 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + C::kNumBars);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int ntile = blockIdx.x, kvh = blockIdx.y, b = blockIdx.z;
-  const int n0 = ntile * kBwdTile;
-  const int diag = p.Nk - p.Nq;  // causal: key j is allowed for query i iff j <= i + diag
-  const int nq_tiles = (p.Nq + kBwdTile - 1) / kBwdTile;
+  BwdSeq sq;
+  if (!bwd_locate(p, blockIdx.x, blockIdx.z, sq)) return;  // varlen: no tile of this index
+  const int kvh = blockIdx.y;
+  const int Nq = sq.nq, Nk = sq.nk;
+  const int n0 = sq.tile * kBwdTile;
+  const int diag = Nk - Nq;  // causal: key j is allowed for query i iff j <= i + diag
+  const int nq_tiles = (Nq + kBwdTile - 1) / kBwdTile;
   int i_lo = 0;
   if (p.causal) {
     const int need = n0 - diag - (kBwdTile - 1);  // first tile whose last query sees key n0
@@ -208,8 +347,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     if (T > 0) {
       mbar_arrive_expect_tx_elect(kv_full, 2 * C::kTileBytes);
       for (int c = 0; c < D / 64; ++c) {
-        tma_load_3d_elect(sK + c * C::kChunkBytes, &tmK, c * 64, kvh, b * p.Nk + n0, kv_full);
-        tma_load_3d_elect(sV + c * C::kChunkBytes, &tmV, c * 64, kvh, b * p.Nk + n0, kv_full);
+        tma_load_3d_elect(sK + c * C::kChunkBytes, &tmK, c * 64, kvh, sq.rowk + n0, kv_full);
+        tma_load_3d_elect(sV + c * C::kChunkBytes, &tmV, c * 64, kvh, sq.rowk + n0, kv_full);
       }
       for (int t = 0; t < T; ++t) {
         const int slot = t & 1;
@@ -218,12 +357,12 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         const int q0 = (i_lo + t % ntq) * kBwdTile;
         mbar_arrive_expect_tx_elect(q_full + slot, 2 * C::kTileBytes + 2 * C::kVecBytes);
         for (int c = 0; c < D / 64; ++c) {
-          tma_load_3d_elect(sQ + slot * C::kTileBytes + c * C::kChunkBytes, &tmQ, c * 64, h, b * p.Nq + q0,
+          tma_load_3d_elect(sQ + slot * C::kTileBytes + c * C::kChunkBytes, &tmQ, c * 64, h, sq.rowq + q0,
                             q_full + slot);
-          tma_load_3d_elect(sDO + slot * C::kTileBytes + c * C::kChunkBytes, &tmDO, c * 64, h, b * p.Nq + q0,
+          tma_load_3d_elect(sDO + slot * C::kTileBytes + c * C::kChunkBytes, &tmDO, c * 64, h, sq.rowq + q0,
                             q_full + slot);
         }
-        const size_t voff = ((size_t)b * p.Hq + h) * p.NqPad + q0;
+        const size_t voff = (size_t)(sq.vec0 + h * sq.vech + q0);
         bulk_load_elect(sVec + (slot * 2 + 0) * kBwdTile, p.lse2 + voff, C::kVecBytes, q_full + slot);
         bulk_load_elect(sVec + (slot * 2 + 1) * kBwdTile, p.dvec + voff, C::kVecBytes, q_full + slot);
       }
@@ -292,7 +431,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     const int r = (warp & 3) * 32 + lane;  // key row of the tile = TMEM lane
     const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
     const int key = n0 + r;
-    const bool key_ok = key < p.Nk;
+    const bool key_ok = key < Nk;
     const float tau = p.tau;
     bool ok = true;
     for (int t = 0; t < T && ok; ++t) {
@@ -371,7 +510,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         const uint32_t src = (D == 128) ? (tmem + lane_off + (wg ? C::kColDP : C::kColS) + 64)
                                         : (tmem + lane_off + C::kColS + 64 + 32 * wg);
         const int q = q0 + r;
-        float* dst = p.dq_acc + (((size_t)b * p.Nq + q) * p.Hq + h) * D + wg * kCols;
+        float* dst = p.dq_acc + (((size_t)sq.rowq + q) * p.Hq + h) * D + wg * kCols;
         uint32_t a0[32], a1[32];
         tmem_ld32(src, a0);
         if (kCols == 64) tmem_ld32(src + 32, a1);
@@ -381,7 +520,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(dq_free);
-        if (q < p.Nq) {
+        if (q < Nq) {
 #pragma unroll
           for (int e = 0; e < 32; e += 4)
             red_add_v4(dst + e, __uint_as_float(a0[e]), __uint_as_float(a0[e + 1]), __uint_as_float(a0[e + 2]),
@@ -399,7 +538,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     // (T is uniform over the CTA, so every warp takes the same path to the collective loads)
     const bool have = T > 0 && ok && warp_wait(acc_done, 0);
     tc_fence_after();
-    __nv_bfloat16* dst = (wg ? p.dk : p.dv) + (((size_t)b * p.Nk + key) * p.Hkv + kvh) * D;
+    __nv_bfloat16* dst = (wg ? p.dk : p.dv) + (((size_t)sq.rowk + key) * p.Hkv + kvh) * D;
     const float mul = wg ? p.scale : 1.f;
 #pragma unroll
     for (int c = 0; c < D / 32; ++c) {
@@ -511,10 +650,13 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + C::kNumBars);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int ntile = blockIdx.x, kvh = blockIdx.y, b = blockIdx.z;
-  const int n0 = ntile * kBwdTile;
-  const int diag = p.Nk - p.Nq;
-  const int nq_tiles = (p.Nq + kBwdQ - 1) / kBwdQ;
+  BwdSeq sq;
+  if (!bwd_locate(p, blockIdx.x, blockIdx.z, sq)) return;  // varlen: no tile of this index
+  const int kvh = blockIdx.y;
+  const int Nq = sq.nq, Nk = sq.nk;
+  const int n0 = sq.tile * kBwdTile;
+  const int diag = Nk - Nq;
+  const int nq_tiles = (Nq + kBwdQ - 1) / kBwdQ;
   int i_lo = 0;
   if (p.causal) {
     const int need = n0 - diag - (kBwdQ - 1);  // first 64-query tile whose last query sees key n0
@@ -560,7 +702,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         if (!mbar_wait(stage_full, tp & 1)) break;
         const int h = kvh * p.G + tp / ntq;
         const int q0 = (i_lo + tp % ntq) * kBwdQ;
-        tma_reduce_add_3d(&tmDQ, sStage, 0, h, b * p.Nq + q0);
+        tma_reduce_add_3d(&tmDQ, sStage, 0, h, sq.rowq + q0);
         bulk_commit_group();
         bulk_wait_group_read0();
         mbar_arrive(stage_free);
@@ -573,8 +715,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     if (T > 0) {
       mbar_arrive_expect_tx_elect(kv_full, 2 * C::kKTile);
       for (int c = 0; c < D / 64; ++c) {
-        tma_load_3d_elect(sK + c * C::kKPanel, &tmK, c * 64, kvh, b * p.Nk + n0, kv_full);
-        tma_load_3d_elect(sV + c * C::kKPanel, &tmV, c * 64, kvh, b * p.Nk + n0, kv_full);
+        tma_load_3d_elect(sK + c * C::kKPanel, &tmK, c * 64, kvh, sq.rowk + n0, kv_full);
+        tma_load_3d_elect(sV + c * C::kKPanel, &tmV, c * 64, kvh, sq.rowk + n0, kv_full);
       }
       for (int t = 0; t < T; ++t) {
         const int slot = t % kBwdSlots;
@@ -583,11 +725,11 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         const int q0 = (i_lo + t % ntq) * kBwdQ;
         mbar_arrive_expect_tx_elect(q_full + slot, 2 * C::kQTile + 2 * C::kVecBytes);
         for (int c = 0; c < D / 64; ++c) {
-          tma_load_3d_elect(sQ + slot * C::kQTile + c * C::kQPanel, &tmQ, c * 64, h, b * p.Nq + q0, q_full + slot);
-          tma_load_3d_elect(sDO + slot * C::kQTile + c * C::kQPanel, &tmDO, c * 64, h, b * p.Nq + q0,
+          tma_load_3d_elect(sQ + slot * C::kQTile + c * C::kQPanel, &tmQ, c * 64, h, sq.rowq + q0, q_full + slot);
+          tma_load_3d_elect(sDO + slot * C::kQTile + c * C::kQPanel, &tmDO, c * 64, h, sq.rowq + q0,
                             q_full + slot);
         }
-        const size_t voff = ((size_t)b * p.Hq + h) * p.NqPad + q0;
+        const size_t voff = (size_t)(sq.vec0 + h * sq.vech + q0);
         bulk_load_elect(sVec + (slot * 2 + 0) * kBwdQ, p.lse2 + voff, C::kVecBytes, q_full + slot);
         bulk_load_elect(sVec + (slot * 2 + 1) * kBwdQ, p.dvec + voff, C::kVecBytes, q_full + slot);
       }
@@ -663,7 +805,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     const int r = (warp & 3) * 32 + lane;  // TMEM lane: key row (S, dP) or d (dQ^T)
     const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
     const int key = n0 + r;
-    const bool key_ok = key < p.Nk;
+    const bool key_ok = key < Nk;
     const float tau = p.tau;
     bool ok = true;
 
@@ -775,7 +917,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     // ---- epilogue: dV (warpgroup 0) and dK = scale * acc (warpgroup 1), rows of this key tile
     const bool have = T > 0 && ok && warp_wait(acc_done, 0);
     tc_fence_after();
-    __nv_bfloat16* dst = (wg ? p.dk : p.dv) + (((size_t)b * p.Nk + key) * p.Hkv + kvh) * D;
+    __nv_bfloat16* dst = (wg ? p.dk : p.dv) + (((size_t)sq.rowk + key) * p.Hkv + kvh) * D;
     const float mul = wg ? p.scale : 1.f;
 #pragma unroll
     for (int c = 0; c < D / 32; ++c) {

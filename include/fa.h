@@ -139,6 +139,28 @@ FA_EXPORT fa_status fa_bwd(const void* q, const void* k, const void* v, const vo
 
 FA_EXPORT size_t fa_bwd_workspace_size(int B, int Hq, int Nq, int d);
 
+/* Backward of fa_fwd on packed variable-length sequences ("FlashAttention-3 (FA-3)", feature
+ * table: variable-length batches; the method is that of fa_bwd, within each sequence).
+ *
+ * Sequence b owns rows [cu_seqlens[b], cu_seqlens[b+1]) of q, o, dout, dq [total, Hq, d] and
+ * of k, v, dk, dv [total, Hkv, d] (bf16); lse [Hq, total] fp32 as fa_fwd wrote it with the same
+ * cu_seqlens.  No attention, and so no gradient, crosses a sequence boundary; causal is
+ * within each sequence.  cu_seqlens: device int32 [B + 1], starting at or above 0, never
+ * decreasing, ending at or below total; rows outside every sequence get dq = 0 and their dk,
+ * dv are not written.  Rows of q, k, v and dout past cu_seqlens[B] are read as padding of
+ * the last sequence's last tile and must hold finite values.  A cu_seqlens that breaks this is found on the device: nothing is
+ * computed and fa_last_device_error reports FA_ERR_INVALID_ARG.
+ * d 64 or 128; pointers 16-byte aligned (lse and cu_seqlens 4-byte aligned).
+ * workspace: at least fa_bwd_varlen_workspace_size(B, Hq, total, d) bytes (tile prefix sums,
+ * two fp32 row vectors padded per sequence to 128-row tiles, an fp32 dq accumulator); its
+ * contents need not be initialised. */
+FA_EXPORT fa_status fa_bwd_varlen(const void* q, const void* k, const void* v, const void* o, const void* dout,
+                                  const float* lse, void* dq, void* dk, void* dv, int B, int Hq, int Hkv, int total,
+                                  int d, float scale, int causal, const int32_t* cu_seqlens, void* workspace,
+                                  size_t workspace_bytes, void* stream);
+
+FA_EXPORT size_t fa_bwd_varlen_workspace_size(int B, int Hq, int total, int d);
+
 /* Split-KV decode: one query token per sequence against its KV cache.
  *
  * q [B, Hq, d] bf16; kcache and vcache [B, Lmax, Hkv, d] bf16; o [B, Hq, d] bf16;
@@ -220,7 +242,8 @@ FA_EXPORT size_t fa_decode_paged_workspace_size(int B, int Hq, int Hkv, int max_
 /* Waits for `stream`, then returns FA_ERR_TIMEOUT if any kernel of this library recorded a
  * device-side timeout since the previous call, else FA_ERR_CUDA if a kernel found its shared
  * memory carve-out too small, else FA_ERR_INVALID_ARG if a kernel recorded an invalid
- * device-side input (a block-table entry out of range), and clears the record; FA_ERR_CUDA
+ * device-side input (a block-table entry out of range, a
+ * cu_seqlens that fa_bwd_varlen cannot use), and clears the record; FA_ERR_CUDA
  * if the stream reports an error; else FA_OK. */
 FA_EXPORT fa_status fa_last_device_error(void* stream);
 

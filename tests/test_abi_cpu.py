@@ -164,6 +164,34 @@ def test_bwd_rejects_before_launch(lib):
     assert fa.fa_bwd_workspace_size(1, 64, 8192, 128) >= 8192 * 64 * 128 * 4
 
 
+def test_bwd_varlen_rejects_before_launch(lib):
+    def st(**kw):
+        a = dict(q=256, k=256, v=256, o=256, do=256, lse=512, dq=256, dk=256, dv=256, B=2, Hq=2, Hkv=1, total=8,
+                 d=128, scale=0.1, causal=1, cu=1024, ws=256, wsb=1 << 30)
+        a.update(kw)
+        return lib.fa_bwd_varlen(a["q"], a["k"], a["v"], a["o"], a["do"], a["lse"], a["dq"], a["dk"], a["dv"],
+                                 a["B"], a["Hq"], a["Hkv"], a["total"], a["d"], ctypes.c_float(a["scale"]),
+                                 a["causal"], a["cu"], a["ws"], a["wsb"], None)
+    assert st(cu=None) == fa.FA_ERR_INVALID_ARG
+    assert st(cu=1026) == fa.FA_ERR_INVALID_ARG      # misaligned cu_seqlens
+    assert st(dv=None) == fa.FA_ERR_INVALID_ARG
+    assert st(q=264) == fa.FA_ERR_INVALID_ARG        # misaligned
+    assert st(total=-1) == fa.FA_ERR_INVALID_ARG
+    assert st(d=96) == fa.FA_ERR_UNSUPPORTED
+    assert st(Hq=3, Hkv=2) == fa.FA_ERR_UNSUPPORTED
+    assert st(scale=float("nan")) == fa.FA_ERR_INVALID_ARG
+    assert st(ws=None) == fa.FA_ERR_WORKSPACE
+    assert st(wsb=fa.fa_bwd_varlen_workspace_size(2, 2, 8, 128) - 1) == fa.FA_ERR_WORKSPACE
+    assert st(B=0) == fa.FA_OK
+    assert st(total=0) == fa.FA_OK
+    assert fa.fa_bwd_varlen_workspace_size(0, 2, 8, 128) == 0
+    # the row vectors hold one 128-row tile per sequence even when every sequence is one row
+    # long (the most tiles per row), next to the fp32 dq accumulator
+    for B, Hq, d in ((1, 1, 64), (16, 32, 128), (1000, 8, 128)):
+        assert fa.fa_bwd_varlen_workspace_size(B, Hq, B, d) >= 2 * Hq * B * 128 * 4 + B * Hq * d * 4
+    assert fa.fa_bwd_varlen_workspace_size(16, 32, 67584, 128) >= 67584 * 32 * 128 * 4
+
+
 def test_fp8_and_packed_reject_before_launch(lib):
     def st8(**kw):
         a = dict(q=256, k=256, v=256, o=256, lse=None, B=1, Hq=2, Hkv=1, Nq=8, Nk=8, d=128, scale=0.1, dq=1.0,
