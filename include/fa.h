@@ -14,7 +14,8 @@
  *              results are merged with the same m/l rule ("FlashAttention-3 (FA-3)",
  *              section 4 "FlashDecoding"; "FlashAttention notes", section 4).
  *   fa_decode_paged  the same decode over a paged cache addressed through a block table.
- *   fa_bwd     the backward of fa_fwd by recomputation from the saved logsumexp.
+ *   fa_bwd     the backward of fa_fwd by recomputation from the saved logsumexp;
+ *              fa_bwd_varlen the same over packed variable-length sequences.
  *   fa_fwd_qkvpacked  fa_fwd reading q, k, v from one packed [.., 3, H, d] tensor.
  *   fa_fwd_fp8 the forward on e4m3 inputs with per-tensor scales.
  *
