@@ -84,10 +84,17 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
 
 
 def _ptr(x) -> Optional[int]:
+    """Device address of a tensor argument (an int is taken as a raw address).  The library
+    reads every tensor as a dense row-major block of device memory, so a host tensor or a
+    strided view is refused here rather than handed to a kernel."""
     if x is None:
         return None
     if isinstance(x, int):
         return x or None
+    if not x.is_cuda:
+        raise ValueError(f"expected a CUDA tensor, got one on {x.device}")
+    if not x.is_contiguous():
+        raise ValueError(f"expected a contiguous tensor, got strides {tuple(x.stride())} for shape {tuple(x.shape)}")
     return x.data_ptr() or None
 
 

@@ -144,6 +144,36 @@ def test_binding_raises_fa_error(lib):
     assert e.value.status == fa.FA_ERR_UNSUPPORTED
 
 
+def test_binding_refuses_host_and_strided_tensors(lib):
+    """The binding hands the library only dense device memory: a host tensor or a strided
+    view raises before any call (the library itself cannot tell a host pointer from a device
+    one)."""
+    import torch
+    host = torch.zeros(1, 8, 2, 64, dtype=torch.bfloat16)
+    with pytest.raises(ValueError, match="CUDA tensor"):
+        fa.fa_fwd(host, 256, 256, 256, None, 1, 2, 1, 8, 8, 64, 0.1, 1, stream=0)
+    with pytest.raises(ValueError, match="CUDA tensor"):
+        fa.forward(host, host, host, stream=0)
+    with pytest.raises(ValueError, match="CUDA tensor"):
+        fa.fa_decode(256, 256, 256, torch.zeros(2, dtype=torch.int32), 256, None, 2, 8, 2, 64, 64, 0.1, 64, 256,
+                     1 << 20, stream=0)
+
+    class FakeStrided:  # a device tensor whose layout is not dense
+        is_cuda = True
+        shape, device = (8, 64), "cuda:0"
+
+        def is_contiguous(self):
+            return False
+
+        def stride(self):
+            return (1, 8)
+
+        def data_ptr(self):
+            raise AssertionError("a strided tensor's address must not be taken")
+    with pytest.raises(ValueError, match="contiguous"):
+        fa.fa_fwd(FakeStrided(), 256, 256, 256, None, 1, 2, 1, 8, 8, 64, 0.1, 1, stream=0)
+
+
 def test_bwd_rejects_before_launch(lib):
     def st(**kw):
         a = dict(q=256, k=256, v=256, o=256, do=256, lse=512, dq=256, dk=256, dv=256, B=1, Hq=2, Hkv=1, Nq=8, Nk=8,
