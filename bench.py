@@ -284,7 +284,9 @@ def run_device(args):
     # ---- paged ragged decode: shuffled pool of 16-token pages, block table, lengths
     wp = PAGED
     pseed = replica_seed(wp["seed"], rank)
-    p_len = paged_lengths(pseed) if do_paged else np.ones(1, np.int64)
+    # the lengths are the workload's shape, the same on every rank (so N ranks do N times the
+    # work of one); the values and the page placement are each rank's own
+    p_len = paged_lengths(wp["seed"]) if do_paged else np.ones(1, np.int64)
     pB = len(p_len)
     pps, pHq, pHkv, pd, psplit = wp["page_size"], wp["Hq"], wp["Hkv"], wp["d"], wp["split"]
     table_np, npages = si.page_layout(pseed, p_len, pps)
@@ -320,7 +322,7 @@ def run_device(args):
 
     if do_bwdv:
         vseed = replica_seed(VARLEN["seed"], rank)
-        v_len = varlen_lengths(vseed)
+        v_len = varlen_lengths(VARLEN["seed"])  # the same lengths on every rank, own values
         v_cu_np = si.cu_seqlens(v_len)
         vT, vB = int(v_cu_np[-1]), len(v_len)
         vHq, vHkv, vd = VARLEN["Hq"], VARLEN["Hkv"], VARLEN["d"]

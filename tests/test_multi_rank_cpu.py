@@ -68,3 +68,13 @@ def test_paged_workload_bytes_follow_lengths():
     lens = bench.paged_lengths(w["seed"])
     assert len(lens) == w["B"] and lens.min() >= w["len_lo"] and lens.max() <= w["len_hi"]
     assert bench.paged_kv_bytes(lens) == 2.0 * lens.sum() * w["Hkv"] * w["d"] * 2
+
+
+def test_varlen_flops_match_the_closed_form():
+    """Causal varlen forward FLOPs: sum over sequences of 4 Hq L^2 d / 2, which for Hq = 32,
+    d = 128 is 8192 L^2 per sequence; the backward counts 2.5 times that."""
+    lens = bench.varlen_lengths(bench.VARLEN["seed"])
+    assert len(lens) == bench.VARLEN["nseq"]
+    assert lens.min() >= bench.VARLEN["len_lo"] and lens.max() <= bench.VARLEN["len_hi"]
+    assert bench.varlen_flops(lens) == float(sum(8192 * int(L) * int(L) for L in lens))
+    assert bench.varlen_flops([5]) == 4 * 32 * 25 * 128 / 2
