@@ -78,3 +78,27 @@ def test_varlen_flops_match_the_closed_form():
     assert lens.min() >= bench.VARLEN["len_lo"] and lens.max() <= bench.VARLEN["len_hi"]
     assert bench.varlen_flops(lens) == float(sum(8192 * int(L) * int(L) for L in lens))
     assert bench.varlen_flops([5]) == 4 * 32 * 25 * 128 / 2
+
+
+def test_reference_arm_prints_one_contract_line():
+    """`bench.py --impl reference` times the oracle on the host and prints one JSON line with
+    the contract's keys; a rank other than 0 prints nothing and exits 0."""
+    import json
+    import os
+    import subprocess
+    import sys
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    cmd = [sys.executable, os.path.join(root, "bench.py"), "--impl", "reference", "--steps", "1", "--warmup", "0",
+           "--cpu-seconds", "1"]
+    out = subprocess.run(cmd, cwd=root, capture_output=True, text=True, timeout=300,
+                         env={**os.environ, "RANK": "0", "WORLD_SIZE": "1"})
+    assert out.returncode == 0, out.stderr[-2000:]
+    lines = [ln for ln in out.stdout.splitlines() if ln.startswith("{")]
+    assert len(lines) == 1
+    j = json.loads(lines[0])
+    assert j["impl"] == "reference" and j["unit"] == "TFLOP/s" and j["higher_is_better"] is True
+    assert j["value"] > 0 and j["cpu_baseline"]["kind"] == "oracle" and j["cpu_baseline"]["cores"] >= 1
+    assert j["e2e"] == {"value": j["value"], "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}
+    other = subprocess.run(cmd, cwd=root, capture_output=True, text=True, timeout=300,
+                           env={**os.environ, "RANK": "1", "WORLD_SIZE": "2"})
+    assert other.returncode == 0 and not other.stdout.strip()
