@@ -98,6 +98,30 @@ def _ptr(x) -> Optional[int]:
     return x.data_ptr() or None
 
 
+def _ptr_i32(x, what: str) -> Optional[int]:
+    """Device address of an int32 index tensor (offsets, lengths, block table): the kernels
+    read these as int32, so another integer width would be misread as other offsets."""
+    if x is not None and not isinstance(x, int) and str(x.dtype) != "torch.int32":
+        raise ValueError(f"{what}: expected an int32 tensor, got {x.dtype}")
+    return _ptr(x)
+
+
+def _expect(t, shape, dtype: str, what: str) -> None:
+    """A caller-provided output must have exactly the shape and dtype the kernels write."""
+    if t is None:
+        return
+    if tuple(t.shape) != tuple(shape) or str(t.dtype) != dtype:
+        raise ValueError(f"{what}: expected {dtype} {tuple(shape)}, got {t.dtype} {tuple(t.shape)}")
+
+
+def _same(what: str, *ts) -> None:
+    """Tensors that the kernels read with one shape and one element type."""
+    a = ts[0]
+    for t in ts[1:]:
+        if tuple(t.shape) != tuple(a.shape) or t.dtype != a.dtype:
+            raise ValueError(f"{what}: shapes/dtypes differ: {tuple(a.shape)} {a.dtype} vs {tuple(t.shape)} {t.dtype}")
+
+
 def _stream(stream) -> Optional[int]:
     if stream is None:
         import torch
@@ -119,7 +143,7 @@ def status_string(status: int) -> str:
 def fa_fwd(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, d, scale, causal, cu_seqlens=None, in_dtype=FA_BF16,
            workspace=None, workspace_bytes=0, stream=None) -> None:
     st = load().fa_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), int(B), int(Hq), int(Hkv), int(Nq), int(Nk),
-                       int(d), float(scale), int(bool(causal)), _ptr(cu_seqlens), int(in_dtype), _ptr(workspace),
+                       int(d), float(scale), int(bool(causal)), _ptr_i32(cu_seqlens, "cu_seqlens"), int(in_dtype), _ptr(workspace),
                        int(workspace_bytes), _stream(stream))
     _check(st, "fa_fwd")
 
@@ -131,7 +155,7 @@ def fa_fwd_workspace_size(B, Hq, Hkv, Nq, Nk, d, in_dtype=FA_BF16, varlen=False)
 
 def fa_decode(q, kcache, vcache, seqlens, o, lse, B, Hq, Hkv, Lmax, d, scale, split_len, workspace,
               workspace_bytes, stream=None) -> None:
-    st = load().fa_decode(_ptr(q), _ptr(kcache), _ptr(vcache), _ptr(seqlens), _ptr(o), _ptr(lse), int(B), int(Hq),
+    st = load().fa_decode(_ptr(q), _ptr(kcache), _ptr(vcache), _ptr_i32(seqlens, "seqlens"), _ptr(o), _ptr(lse), int(B), int(Hq),
                           int(Hkv), int(Lmax), int(d), float(scale), int(split_len), _ptr(workspace),
                           int(workspace_bytes), _stream(stream))
     _check(st, "fa_decode")
@@ -142,7 +166,7 @@ def fa_decode_noalloc(q, kcache, vcache, seqlens, o, lse, B, Hq, Hkv, Lmax, d, s
     """fa_decode with its scratch in the library's static device array (no allocation).
     For callers that cannot allocate device memory; calls that overlap on the GPU race, and
     the first call on a device should come before any stream capture (see include/fa.h)."""
-    st = load().fa_decode_noalloc(_ptr(q), _ptr(kcache), _ptr(vcache), _ptr(seqlens), _ptr(o), _ptr(lse), int(B),
+    st = load().fa_decode_noalloc(_ptr(q), _ptr(kcache), _ptr(vcache), _ptr_i32(seqlens, "seqlens"), _ptr(o), _ptr(lse), int(B),
                                   int(Hq), int(Hkv), int(Lmax), int(d), float(scale), int(split_len),
                                   _stream(stream))
     _check(st, "fa_decode_noalloc")
@@ -154,7 +178,7 @@ def fa_decode_workspace_size(B, Hq, Lmax, d, split_len) -> int:
 
 def fa_decode_paged(q, k_pages, v_pages, block_table, seqlens, o, lse, B, Hq, Hkv, num_pages, page_size,
                     max_pages_per_seq, d, scale, split_len, workspace, workspace_bytes, stream=None) -> None:
-    st = load().fa_decode_paged(_ptr(q), _ptr(k_pages), _ptr(v_pages), _ptr(block_table), _ptr(seqlens), _ptr(o),
+    st = load().fa_decode_paged(_ptr(q), _ptr(k_pages), _ptr(v_pages), _ptr_i32(block_table, "block_table"), _ptr_i32(seqlens, "seqlens"), _ptr(o),
                                 _ptr(lse), int(B), int(Hq), int(Hkv), int(num_pages), int(page_size),
                                 int(max_pages_per_seq), int(d), float(scale), int(split_len), _ptr(workspace),
                                 int(workspace_bytes), _stream(stream))
@@ -180,7 +204,7 @@ def fa_fwd_fp8_workspace_size(B, Hkv, Nk, d) -> int:
 
 def fa_fwd_qkvpacked(qkv, o, lse, B, H, N, d, scale, causal, cu_seqlens=None, stream=None) -> None:
     st = load().fa_fwd_qkvpacked(_ptr(qkv), _ptr(o), _ptr(lse), int(B), int(H), int(N), int(d), float(scale),
-                                 int(bool(causal)), _ptr(cu_seqlens), _stream(stream))
+                                 int(bool(causal)), _ptr_i32(cu_seqlens, "cu_seqlens"), _stream(stream))
     _check(st, "fa_fwd_qkvpacked")
 
 
@@ -200,7 +224,7 @@ def fa_bwd_varlen(q, k, v, o, dout, lse, dq, dk, dv, B, Hq, Hkv, total, d, scale
                   workspace_bytes, stream=None) -> None:
     st = load().fa_bwd_varlen(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(dout), _ptr(lse), _ptr(dq), _ptr(dk),
                               _ptr(dv), int(B), int(Hq), int(Hkv), int(total), int(d), float(scale),
-                              int(bool(causal)), _ptr(cu_seqlens), _ptr(workspace), int(workspace_bytes),
+                              int(bool(causal)), _ptr_i32(cu_seqlens, "cu_seqlens"), _ptr(workspace), int(workspace_bytes),
                               _stream(stream))
     _check(st, "fa_bwd_varlen")
 
@@ -231,6 +255,9 @@ def forward(q, k, v, causal=False, scale=None, cu_seqlens=None, out=None, lse=No
     give fp32 O.  Outputs and workspace are allocated with torch unless passed in."""
     import torch
     varlen = cu_seqlens is not None
+    _same("k, v", k, v)
+    if q.dtype != k.dtype or q.shape[-1] != k.shape[-1] or q.dim() != k.dim():
+        raise ValueError(f"q {q.dtype} {tuple(q.shape)} does not match k {k.dtype} {tuple(k.shape)}")
     if varlen:
         total, Hq, d = q.shape
         Hkv = k.shape[1]
@@ -243,6 +270,8 @@ def forward(q, k, v, causal=False, scale=None, cu_seqlens=None, out=None, lse=No
     in_dtype = (FA_TF32 if tf32 else FA_F32) if q.dtype == torch.float32 else FA_BF16
     if scale is None:
         scale = d ** -0.5
+    _expect(out, q.shape, "torch.bfloat16" if in_dtype == FA_BF16 else "torch.float32", "out")
+    _expect(lse, lse_shape, "torch.float32", "lse")
     if out is None:
         out = torch.empty(q.shape, dtype=torch.bfloat16 if in_dtype == FA_BF16 else torch.float32, device=q.device)
     if lse is None:
@@ -260,9 +289,12 @@ def decode(q, kcache, vcache, seqlens=None, scale=None, split_len=1024, out=None
     """O [B,Hq,d], lse [B,Hq] for one query token per sequence over caches [B,Lmax,Hkv,d]."""
     import torch
     B, Hq, d = q.shape
+    _same("kcache, vcache", kcache, vcache)
     Lmax, Hkv = kcache.shape[1], kcache.shape[2]
     if scale is None:
         scale = d ** -0.5
+    _expect(out, (B, Hq, d), "torch.bfloat16", "out")
+    _expect(lse, (B, Hq), "torch.float32", "lse")
     if out is None:
         out = torch.empty((B, Hq, d), dtype=torch.bfloat16, device=q.device)
     if lse is None:
@@ -283,10 +315,15 @@ def decode_paged(q, k_pages, v_pages, block_table, seqlens, scale=None, split_le
     counters); calls leave it ready for the next call."""
     import torch
     B, Hq, d = q.shape
+    _same("k_pages, v_pages", k_pages, v_pages)
     num_pages, page_size, Hkv = k_pages.shape[0], k_pages.shape[1], k_pages.shape[2]
+    if block_table.dim() != 2 or block_table.shape[0] != B:
+        raise ValueError(f"block_table: expected [B={B}, max_pages], got {tuple(block_table.shape)}")
     maxp = block_table.shape[1]
     if scale is None:
         scale = d ** -0.5
+    _expect(out, (B, Hq, d), "torch.bfloat16", "out")
+    _expect(lse, (B, Hq), "torch.float32", "lse")
     if out is None:
         out = torch.empty((B, Hq, d), dtype=torch.bfloat16, device=q.device)
     if lse is None:
@@ -303,7 +340,10 @@ def backward(q, k, v, o, lse, dout, causal=False, scale=None, workspace=None, st
     """dq, dk, dv for q [B,Nq,Hq,d], k/v [B,Nk,Hkv,d], the forward's o and lse, and dout."""
     import torch
     B, Nq, Hq, d = q.shape
+    _same("q, o, dout", q, o, dout)
+    _same("k, v", k, v)
     Nk, Hkv = k.shape[1], k.shape[2]
+    _expect(lse, (B, Hq, Nq), "torch.float32", "lse")
     if scale is None:
         scale = d ** -0.5
     dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
@@ -319,8 +359,11 @@ def backward_varlen(q, k, v, o, lse, dout, cu_seqlens, causal=False, scale=None,
     from the varlen forward, cu_seqlens int32 [B+1] on the device."""
     import torch
     total, Hq, d = q.shape
+    _same("q, o, dout", q, o, dout)
+    _same("k, v", k, v)
     Hkv = k.shape[1]
     B = cu_seqlens.numel() - 1
+    _expect(lse, (Hq, total), "torch.float32", "lse")
     if scale is None:
         scale = d ** -0.5
     dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)

@@ -174,6 +174,40 @@ def test_binding_refuses_host_and_strided_tensors(lib):
         fa.fa_fwd(FakeStrided(), 256, 256, 256, None, 1, 2, 1, 8, 8, 64, 0.1, 1, stream=0)
 
 
+def test_binding_checks_index_types_and_output_shapes(lib):
+    """Index tensors must be int32 and caller-provided outputs must match what the kernels
+    write; the binding says so before anything is called."""
+    import torch
+    bf = torch.bfloat16
+    q = torch.zeros(2, 16, 4, 64, dtype=bf)
+    k = torch.zeros(2, 16, 2, 64, dtype=bf)
+    with pytest.raises(ValueError, match="int32"):
+        fa.fa_fwd(256, 256, 256, 256, None, 2, 4, 2, 16, 16, 64, 0.1, 1, cu_seqlens=torch.zeros(3, dtype=torch.int64),
+                  stream=0)
+    with pytest.raises(ValueError, match="int32"):
+        fa.fa_decode(256, 256, 256, torch.zeros(2, dtype=torch.int64), 256, None, 2, 8, 2, 64, 64, 0.1, 64, 256,
+                     1 << 20, stream=0)
+    with pytest.raises(ValueError, match="int32"):
+        fa.fa_decode_paged(256, 256, 256, torch.zeros(2, 4, dtype=torch.int64), None, 256, None, 2, 8, 2, 16, 16,
+                           4, 64, 0.1, 64, 256, 1 << 20, stream=0)
+    with pytest.raises(ValueError, match="out"):
+        fa.forward(q, k, k, out=torch.zeros(2, 16, 4, 64, dtype=torch.float32), stream=0)
+    with pytest.raises(ValueError, match="lse"):
+        fa.forward(q, k, k, lse=torch.zeros(2, 16, 4, dtype=torch.float32), stream=0)
+    with pytest.raises(ValueError, match="k, v"):
+        fa.forward(q, k, torch.zeros(2, 15, 2, 64, dtype=bf), stream=0)
+    with pytest.raises(ValueError, match="does not match"):
+        fa.forward(q, k.float(), k.float(), stream=0)
+    with pytest.raises(ValueError, match="lse"):
+        fa.backward(q, k, k, q, torch.zeros(2, 4, 15, dtype=torch.float32), q, stream=0)
+    with pytest.raises(ValueError, match="q, o, dout"):
+        fa.backward(q, k, k, q.float(), torch.zeros(2, 4, 16, dtype=torch.float32), q, stream=0)
+    with pytest.raises(ValueError, match="block_table"):
+        fa.decode_paged(torch.zeros(2, 4, 64, dtype=bf), torch.zeros(8, 16, 2, 64, dtype=bf),
+                        torch.zeros(8, 16, 2, 64, dtype=bf), torch.zeros(3, 4, dtype=torch.int32),
+                        torch.zeros(2, dtype=torch.int32), stream=0)
+
+
 def test_bwd_rejects_before_launch(lib):
     def st(**kw):
         a = dict(q=256, k=256, v=256, o=256, do=256, lse=512, dq=256, dk=256, dv=256, B=1, Hq=2, Hkv=1, Nq=8, Nk=8,
