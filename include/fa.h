@@ -147,10 +147,11 @@ FA_EXPORT size_t fa_bwd_workspace_size(int B, int Hq, int Nq, int d);
  * of k, v, dk, dv [total, Hkv, d] (bf16); lse [Hq, total] fp32 as fa_fwd wrote it with the same
  * cu_seqlens.  No attention, and so no gradient, crosses a sequence boundary; causal is
  * within each sequence.  cu_seqlens: device int32 [B + 1], starting at or above 0, never
- * decreasing, ending at or below total; rows outside every sequence get dq = 0 and their dk,
- * dv are not written.  Rows of q, k, v and dout past cu_seqlens[B] are read as padding of
- * the last sequence's last tile and must hold finite values.  A cu_seqlens that breaks this is found on the device: nothing is
- * computed and fa_last_device_error reports FA_ERR_INVALID_ARG.
+ * decreasing, ending at or below total; a cu_seqlens that breaks this is found on the
+ * device: nothing is computed and fa_last_device_error reports FA_ERR_INVALID_ARG.  Rows
+ * outside every sequence get dq = 0 and their dk, dv are not written; rows of q, k, v and
+ * dout past cu_seqlens[B] are read as padding of the last sequence's last tile and must hold
+ * finite values.
  * d 64 or 128; pointers 16-byte aligned (lse and cu_seqlens 4-byte aligned).
  * workspace: at least fa_bwd_varlen_workspace_size(B, Hq, total, d) bytes (tile prefix sums,
  * two fp32 row vectors padded per sequence to 128-row tiles, an fp32 dq accumulator); its
