@@ -122,6 +122,13 @@ def _same(what: str, *ts) -> None:
             raise ValueError(f"{what}: shapes/dtypes differ: {tuple(a.shape)} {a.dtype} vs {tuple(t.shape)} {t.dtype}")
 
 
+def _bf16(what: str, *ts) -> None:
+    """Paths that read bf16 only (the backward, the decodes)."""
+    for t in ts:
+        if str(t.dtype) != "torch.bfloat16":
+            raise ValueError(f"{what}: expected bf16 tensors, got {t.dtype}")
+
+
 def _stream(stream) -> Optional[int]:
     if stream is None:
         import torch
@@ -290,6 +297,7 @@ def decode(q, kcache, vcache, seqlens=None, scale=None, split_len=1024, out=None
     import torch
     B, Hq, d = q.shape
     _same("kcache, vcache", kcache, vcache)
+    _bf16("decode", q, kcache)
     Lmax, Hkv = kcache.shape[1], kcache.shape[2]
     if scale is None:
         scale = d ** -0.5
@@ -316,6 +324,7 @@ def decode_paged(q, k_pages, v_pages, block_table, seqlens, scale=None, split_le
     import torch
     B, Hq, d = q.shape
     _same("k_pages, v_pages", k_pages, v_pages)
+    _bf16("decode_paged", q, k_pages)
     num_pages, page_size, Hkv = k_pages.shape[0], k_pages.shape[1], k_pages.shape[2]
     if block_table.dim() != 2 or block_table.shape[0] != B:
         raise ValueError(f"block_table: expected [B={B}, max_pages], got {tuple(block_table.shape)}")
@@ -342,6 +351,7 @@ def backward(q, k, v, o, lse, dout, causal=False, scale=None, workspace=None, st
     B, Nq, Hq, d = q.shape
     _same("q, o, dout", q, o, dout)
     _same("k, v", k, v)
+    _bf16("backward", q, k)
     Nk, Hkv = k.shape[1], k.shape[2]
     _expect(lse, (B, Hq, Nq), "torch.float32", "lse")
     if scale is None:
@@ -361,6 +371,7 @@ def backward_varlen(q, k, v, o, lse, dout, cu_seqlens, causal=False, scale=None,
     total, Hq, d = q.shape
     _same("q, o, dout", q, o, dout)
     _same("k, v", k, v)
+    _bf16("backward_varlen", q, k)
     Hkv = k.shape[1]
     B = cu_seqlens.numel() - 1
     _expect(lse, (Hq, total), "torch.float32", "lse")

@@ -202,6 +202,11 @@ def test_binding_checks_index_types_and_output_shapes(lib):
         fa.backward(q, k, k, q, torch.zeros(2, 4, 15, dtype=torch.float32), q, stream=0)
     with pytest.raises(ValueError, match="q, o, dout"):
         fa.backward(q, k, k, q.float(), torch.zeros(2, 4, 16, dtype=torch.float32), q, stream=0)
+    with pytest.raises(ValueError, match="bf16"):
+        qf, kf = q.float(), k.float()
+        fa.backward(qf, kf, kf, qf, torch.zeros(2, 4, 16, dtype=torch.float32), qf, stream=0)
+    with pytest.raises(ValueError, match="bf16"):
+        fa.decode(torch.zeros(2, 4, 64), torch.zeros(2, 32, 2, 64), torch.zeros(2, 32, 2, 64), stream=0)
     with pytest.raises(ValueError, match="block_table"):
         fa.decode_paged(torch.zeros(2, 4, 64, dtype=bf), torch.zeros(8, 16, 2, 64, dtype=bf),
                         torch.zeros(8, 16, 2, 64, dtype=bf), torch.zeros(3, 4, dtype=torch.int32),
