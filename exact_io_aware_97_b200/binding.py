@@ -122,6 +122,19 @@ def _same(what: str, *ts) -> None:
             raise ValueError(f"{what}: shapes/dtypes differ: {tuple(a.shape)} {a.dtype} vs {tuple(t.shape)} {t.dtype}")
 
 
+def _require(what: str, ok: bool, expected: str) -> None:
+    """A relation between tensors that the kernels rely on: they size every read from q's
+    batch and head dimension, so a smaller k or cache would be read past its end."""
+    if not ok:
+        raise ValueError(f"{what}: expected {expected}")
+
+
+def _lengths(seqlens, B: int, what: str) -> None:
+    """Per-sequence lengths are read as B int32 entries."""
+    if seqlens is not None and not isinstance(seqlens, int):
+        _require(what, seqlens.dim() == 1 and seqlens.numel() == B, f"{B} entries, got shape {tuple(seqlens.shape)}")
+
+
 def _bf16(what: str, *ts) -> None:
     """Paths that read bf16 only (the backward, the decodes)."""
     for t in ts:
@@ -266,14 +279,21 @@ def forward(q, k, v, causal=False, scale=None, cu_seqlens=None, out=None, lse=No
     if q.dtype != k.dtype or q.shape[-1] != k.shape[-1] or q.dim() != k.dim():
         raise ValueError(f"q {q.dtype} {tuple(q.shape)} does not match k {k.dtype} {tuple(k.shape)}")
     if varlen:
+        _require("q", q.dim() == 3, f"packed [total, Hq, d] with cu_seqlens, got shape {tuple(q.shape)}")
         total, Hq, d = q.shape
         Hkv = k.shape[1]
+        _require("k", k.shape[0] == total, f"{total} packed rows like q, got {k.shape[0]}")
+        _require("cu_seqlens", cu_seqlens.dim() == 1 and cu_seqlens.numel() >= 2,
+                 f"[B + 1] offsets, got shape {tuple(cu_seqlens.shape)}")
         B, Nq, Nk = cu_seqlens.numel() - 1, total, total
         lse_shape = (Hq, total)
     else:
+        _require("q", q.dim() == 4, f"[B, Nq, Hq, d], got shape {tuple(q.shape)}")
         B, Nq, Hq, d = q.shape
         Nk, Hkv = k.shape[1], k.shape[2]
+        _require("k", k.shape[0] == B, f"batch {B} like q, got {k.shape[0]}")
         lse_shape = (B, Hq, Nq)
+    _require("heads", Hkv > 0 and Hq % Hkv == 0, f"Hq ({Hq}) a multiple of Hkv ({Hkv})")
     in_dtype = (FA_TF32 if tf32 else FA_F32) if q.dtype == torch.float32 else FA_BF16
     if scale is None:
         scale = d ** -0.5
@@ -295,10 +315,15 @@ def decode(q, kcache, vcache, seqlens=None, scale=None, split_len=1024, out=None
            stream=None):
     """O [B,Hq,d], lse [B,Hq] for one query token per sequence over caches [B,Lmax,Hkv,d]."""
     import torch
+    _require("q", q.dim() == 3, f"[B, Hq, d], got shape {tuple(q.shape)}")
     B, Hq, d = q.shape
     _same("kcache, vcache", kcache, vcache)
     _bf16("decode", q, kcache)
+    _require("kcache", kcache.dim() == 4 and kcache.shape[0] == B and kcache.shape[3] == d,
+             f"[B={B}, Lmax, Hkv, d={d}], got shape {tuple(kcache.shape)}")
     Lmax, Hkv = kcache.shape[1], kcache.shape[2]
+    _require("heads", Hkv > 0 and Hq % Hkv == 0, f"Hq ({Hq}) a multiple of Hkv ({Hkv})")
+    _lengths(seqlens, B, "seqlens")
     if scale is None:
         scale = d ** -0.5
     _expect(out, (B, Hq, d), "torch.bfloat16", "out")
@@ -322,10 +347,15 @@ def decode_paged(q, k_pages, v_pages, block_table, seqlens, scale=None, split_le
     seqlens [B] (int32).  A workspace passed in must have been zero-filled once (its arrival
     counters); calls leave it ready for the next call."""
     import torch
+    _require("q", q.dim() == 3, f"[B, Hq, d], got shape {tuple(q.shape)}")
     B, Hq, d = q.shape
     _same("k_pages, v_pages", k_pages, v_pages)
     _bf16("decode_paged", q, k_pages)
+    _require("k_pages", k_pages.dim() == 4 and k_pages.shape[3] == d,
+             f"[num_pages, page_size, Hkv, d={d}], got shape {tuple(k_pages.shape)}")
     num_pages, page_size, Hkv = k_pages.shape[0], k_pages.shape[1], k_pages.shape[2]
+    _require("heads", Hkv > 0 and Hq % Hkv == 0, f"Hq ({Hq}) a multiple of Hkv ({Hkv})")
+    _lengths(seqlens, B, "seqlens")
     if block_table.dim() != 2 or block_table.shape[0] != B:
         raise ValueError(f"block_table: expected [B={B}, max_pages], got {tuple(block_table.shape)}")
     maxp = block_table.shape[1]
@@ -348,11 +378,15 @@ def decode_paged(q, k_pages, v_pages, block_table, seqlens, scale=None, split_le
 def backward(q, k, v, o, lse, dout, causal=False, scale=None, workspace=None, stream=None):
     """dq, dk, dv for q [B,Nq,Hq,d], k/v [B,Nk,Hkv,d], the forward's o and lse, and dout."""
     import torch
+    _require("q", q.dim() == 4, f"[B, Nq, Hq, d], got shape {tuple(q.shape)}")
     B, Nq, Hq, d = q.shape
     _same("q, o, dout", q, o, dout)
     _same("k, v", k, v)
     _bf16("backward", q, k)
+    _require("k", k.dim() == 4 and k.shape[0] == B and k.shape[3] == d,
+             f"[B={B}, Nk, Hkv, d={d}], got shape {tuple(k.shape)}")
     Nk, Hkv = k.shape[1], k.shape[2]
+    _require("heads", Hkv > 0 and Hq % Hkv == 0, f"Hq ({Hq}) a multiple of Hkv ({Hkv})")
     _expect(lse, (B, Hq, Nq), "torch.float32", "lse")
     if scale is None:
         scale = d ** -0.5
@@ -368,11 +402,17 @@ def backward_varlen(q, k, v, o, lse, dout, cu_seqlens, causal=False, scale=None,
     """dq, dk, dv for packed sequences: q, o, dout [total,Hq,d], k/v [total,Hkv,d], lse [Hq,total]
     from the varlen forward, cu_seqlens int32 [B+1] on the device."""
     import torch
+    _require("q", q.dim() == 3, f"packed [total, Hq, d], got shape {tuple(q.shape)}")
     total, Hq, d = q.shape
     _same("q, o, dout", q, o, dout)
     _same("k, v", k, v)
     _bf16("backward_varlen", q, k)
+    _require("k", k.dim() == 3 and k.shape[0] == total and k.shape[2] == d,
+             f"[total={total}, Hkv, d={d}], got shape {tuple(k.shape)}")
+    _require("cu_seqlens", cu_seqlens.dim() == 1 and cu_seqlens.numel() >= 2,
+             f"[B + 1] offsets, got shape {tuple(cu_seqlens.shape)}")
     Hkv = k.shape[1]
+    _require("heads", Hkv > 0 and Hq % Hkv == 0, f"Hq ({Hq}) a multiple of Hkv ({Hkv})")
     B = cu_seqlens.numel() - 1
     _expect(lse, (Hq, total), "torch.float32", "lse")
     if scale is None:
@@ -390,11 +430,13 @@ def forward_qkvpacked(qkv, causal=False, scale=None, cu_seqlens=None):
     """O, lse for qkv [B,N,3,H,d] (or [total,3,H,d] with cu_seqlens), bf16."""
     import torch
     if cu_seqlens is not None:
+        _require("qkv", qkv.dim() == 4 and qkv.shape[1] == 3, f"[total, 3, H, d], got shape {tuple(qkv.shape)}")
         total, _, H, d = qkv.shape
         B, N = cu_seqlens.numel() - 1, total
         out = torch.empty((total, H, d), dtype=torch.bfloat16, device=qkv.device)
         lse = torch.empty((H, total), dtype=torch.float32, device=qkv.device)
     else:
+        _require("qkv", qkv.dim() == 5 and qkv.shape[2] == 3, f"[B, N, 3, H, d], got shape {tuple(qkv.shape)}")
         B, N, _, H, d = qkv.shape
         out = torch.empty((B, N, H, d), dtype=torch.bfloat16, device=qkv.device)
         lse = torch.empty((B, H, N), dtype=torch.float32, device=qkv.device)
@@ -407,8 +449,13 @@ def forward_qkvpacked(qkv, causal=False, scale=None, cu_seqlens=None):
 def forward_fp8(q8, k8, v8, descale_q, descale_k, descale_v, causal=False, scale=None, workspace=None):
     """O (bf16), lse for e4m3 q8 [B,Nq,Hq,128], k8/v8 [B,Nk,Hkv,128] (uint8 or float8 tensors)."""
     import torch
+    _require("q8", q8.dim() == 4, f"[B, Nq, Hq, d], got shape {tuple(q8.shape)}")
     B, Nq, Hq, d = q8.shape
+    _same("k8, v8", k8, v8)
+    _require("k8", k8.dim() == 4 and k8.shape[0] == B and k8.shape[3] == d,
+             f"[B={B}, Nk, Hkv, d={d}], got shape {tuple(k8.shape)}")
     Nk, Hkv = k8.shape[1], k8.shape[2]
+    _require("heads", Hkv > 0 and Hq % Hkv == 0, f"Hq ({Hq}) a multiple of Hkv ({Hkv})")
     if scale is None:
         scale = d ** -0.5
     o = torch.empty((B, Nq, Hq, d), dtype=torch.bfloat16, device=q8.device)

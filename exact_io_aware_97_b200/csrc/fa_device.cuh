@@ -223,6 +223,13 @@ __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16
       : "memory");
 }
 
+// 8 consecutive 32-bit columns of this thread's TMEM lane.
+__device__ __forceinline__ void tmem_st8(uint32_t taddr, const uint32_t (&r)[8]) {
+  asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"r"(taddr), "r"(r[0]),
+               "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7])
+               : "memory");
+}
+
 // ---------------------------------------------------------------- UMMA descriptors
 // Shared-memory matrix descriptor (sm_100 format): start address, leading and stride
 // byte offsets (all >> 4), version 1 at bit 46, base offset 0, layout type at bits 61..63
@@ -304,7 +311,10 @@ __device__ __forceinline__ void red_add_v4(float* addr, float a, float b, float 
 // ---------------------------------------------------------------- one-lane issue from a converged warp
 // The issuing roles run converged on all 32 lanes (so descriptors and coordinates are
 // warp-uniform) and let elect.sync pick the single lane that issues each operation.
+// Fast path: one try_wait by every lane and one vote (~40 cycles when the phase is already
+// complete, which the MMA warp sees most of the time); the bounded loop only when it is not.
 __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity) {
+  if (__all_sync(0xffffffffu, mbar_try_wait(bar, parity))) return true;
   return __all_sync(0xffffffffu, mbar_wait(bar, parity));
 }
 
@@ -362,6 +372,57 @@ __device__ __forceinline__ void umma_ts_tf32_elect(uint32_t d_tmem, uint32_t a_t
       : "memory");
 }
 
+// True on exactly one lane of a converged warp (the same lane every time for a full warp),
+// for a block of tcgen05 instructions that one thread issues: descriptors and coordinates
+// stay warp-uniform values and only the issue itself is predicated.
+__device__ __forceinline__ bool elect_one_lane() {
+  uint32_t e;
+  asm volatile("{\n\t.reg .pred p;\n\t.reg .b32 r;\n\telect.sync r|p, 0xffffffff;\n\tselp.u32 %0, 1, 0, p;\n\t}"
+               : "=r"(e));
+  return e != 0;
+}
+
+// One-thread MMA issue by operand kind: 0 = kind::f16 (bf16 operands), 1 = kind::f8f6f4
+// (e4m3), 2 = kind::tf32.  SS: A and B from shared-memory descriptors; TS: A from TMEM.
+template <int KIND>
+__device__ __forceinline__ void mma_ss(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                       uint32_t accumulate) {
+  if constexpr (KIND == 1)
+    asm volatile("{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+                 "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+                 "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+                 : "memory");
+  else if constexpr (KIND == 2)
+    asm volatile("{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+                 "tcgen05.mma.cta_group::1.kind::tf32 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+                 "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+                 : "memory");
+  else
+    asm volatile("{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+                 "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+                 "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+                 : "memory");
+}
+template <int KIND>
+__device__ __forceinline__ void mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
+                                       uint32_t accumulate) {
+  if constexpr (KIND == 1)
+    asm volatile("{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+                 "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+                 "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+                 : "memory");
+  else if constexpr (KIND == 2)
+    asm volatile("{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+                 "tcgen05.mma.cta_group::1.kind::tf32 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+                 "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+                 : "memory");
+  else
+    asm volatile("{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+                 "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+                 "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+                 : "memory");
+}
+
 __device__ __forceinline__ void umma_commit_elect(uint64_t* bar) {
   asm volatile(
       "{\n\t.reg .pred e;\n\t.reg .b32 r;\n\telect.sync r|e, 0xffffffff;\n\t"
@@ -411,22 +472,14 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   return *reinterpret_cast<uint32_t*>(&v);
 }
 
-// Same rounding (to nearest, ties to even) done with integer operations instead of the
-// conversion unit, for finite values: add 0x7FFF plus the lowest kept bit, keep the top half.
-__device__ __forceinline__ uint32_t pack_bf16x2_int(float lo, float hi) {
-  uint32_t a = __float_as_uint(lo), b = __float_as_uint(hi);
-  a += 0x7FFFu + ((a >> 16) & 1u);
-  b += 0x7FFFu + ((b >> 16) & 1u);
-  return __byte_perm(a, b, 0x7632);
+// Two floats to e4m3 (round to nearest even, saturating) in the low / high 16 bits of a
+// word, x0 in the lower byte: a word holds four consecutive keys, lowest key first.
+__device__ __forceinline__ uint32_t pack_e4m3x2_lo(float x0, float x1) {
+  uint16_t v;
+  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(v) : "f"(x1), "f"(x0));
+  return (uint32_t)v;
 }
-
-// Four floats to e4m3 (round to nearest even, saturating), packed with x0 in the lowest byte.
-__device__ __forceinline__ uint32_t pack_e4m3x4(float x0, float x1, float x2, float x3) {
-  uint16_t lo, hi;
-  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(lo) : "f"(x1), "f"(x0));
-  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(hi) : "f"(x3), "f"(x2));
-  return (uint32_t)lo | ((uint32_t)hi << 16);
-}
+__device__ __forceinline__ uint32_t pack_e4m3x2_hi(float x0, float x1) { return pack_e4m3x2_lo(x0, x1) << 16; }
 
 __device__ __forceinline__ float fmax3(float a, float b, float c) {
   float d;
@@ -452,34 +505,6 @@ __device__ __forceinline__ uint64_t f2_add(uint64_t a, uint64_t b) {
   uint64_t d;
   asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
   return d;
-}
-
-// 2^x for two finite x >= -125 on the FMA pipe instead of the special-function unit.
-// Method: Cody-Waite style split x = n + f with n = round(x) (adding and subtracting
-// 1.5 * 2^23) and f in [-1/2, 1/2]; 2^f from a degree-3 polynomial whose coefficients were
-// fitted here by the Remez exchange algorithm on the relative error (csrc/exp2_poly.py;
-// max relative error 7.5e-5); 2^n is applied by adding n to the exponent field.
-constexpr float kExp2C0 = 0.9999280571937561f;
-constexpr float kExp2C1 = 0.6932609677314758f;
-constexpr float kExp2C2 = 0.2426111251115799f;
-constexpr float kExp2C3 = 0.0551716685295105f;
-__device__ __forceinline__ void exp2_poly_x2(float x0, float x1, float& y0, float& y1) {
-  const uint64_t magic = f2(12582912.0f, 12582912.0f);
-  const uint64_t neg_magic = f2(-12582912.0f, -12582912.0f);
-  const uint64_t neg_one = f2(-1.0f, -1.0f);
-  const uint64_t x = f2(fmaxf(x0, -125.0f), fmaxf(x1, -125.0f));
-  const uint64_t t = f2_add(x, magic);       // n sits in the low mantissa bits of t
-  const uint64_t nf = f2_add(t, neg_magic);  // n as a float
-  const uint64_t fr = f2_fma(nf, neg_one, x);
-  uint64_t q = f2_fma(fr, f2(kExp2C3, kExp2C3), f2(kExp2C2, kExp2C2));
-  q = f2_fma(q, fr, f2(kExp2C1, kExp2C1));
-  q = f2_fma(q, fr, f2(kExp2C0, kExp2C0));
-  float q0, q1, t0, t1;
-  f2_split(q, q0, q1);
-  f2_split(t, t0, t1);
-  // (t_bits << 23) keeps only n << 23: the bits of 1.5 * 2^23 above bit 8 shift out.
-  y0 = __uint_as_float(__float_as_uint(q0) + (__float_as_uint(t0) << 23));
-  y1 = __uint_as_float(__float_as_uint(q1) + (__float_as_uint(t1) << 23));
 }
 
 }  // namespace fa

@@ -14,7 +14,7 @@
 //   warp  8     tcgen05.mma issuer and TMEM owner
 //   warp  9     TMA producer
 //   warps 10-11 idle (they complete the control warpgroup for the register split)
-// The issuing warps run converged and let one elected lane issue each instruction.
+// The issuing warps run converged and let one elected lane issue each group of instructions.
 // A work unit is 256 query rows (two 128-row tiles) of one (sequence, query head).  Units
 // are ordered longest-first (causal cost grows with the query tile index) and dealt to
 // CTAs in a snake order.  K and V tiles (128 keys each) flow through a shared-memory ring
@@ -27,6 +27,10 @@
 // rescaled lazily: the reference max m only moves when the tile max exceeds it by more than
 // 8 (a factor 256), which is exact because O and l always share the same reference
 // ("LLM basics", chapter 3 section 1: subtracting any constant leaves softmax unchanged).
+// Once a row has a reference, its exponentials start right after the scores are loaded and
+// the tile max, formed alongside, only confirms before publishing that no row moved past
+// the threshold (else the tile is redone against the new max), so the max is off the
+// critical path S(j) -> P(j) -> O += P V -> S(j+1) of each tile.
 #pragma once
 
 #include "fa_device.cuh"
@@ -51,17 +55,20 @@ constexpr int kFwdThreads = 384;
 // Register split by warpgroup, set with setmaxnreg after the common prologue.  The launch
 // gives 384 threads x 168 registers = 64512; softmax warpgroups take 2 x 128 x 208 and the
 // control warpgroup (MMA, TMA, two idle warps) 128 x 88, the same total (and the same per
-// SM sub-partition: two softmax warps and one control warp each).
+// SM sub-partition: two softmax warps and one control warp each).  (A fourth warpgroup
+// for the epilogue leaves the softmax 192 registers at most, which spills: measured slower.)
 constexpr int kSoftmaxRegs = 208;
 constexpr int kControlRegs = 88;
 constexpr int kMaxVarlenB = 1024;
 constexpr int kMaxVarlenT = 1024;
 constexpr float kRescaleThreshold = 8.0f;
-// Column pairs (of each group of 8) whose 2^x runs on the FMA pipe in unmasked tiles, and
-// pairs packed to bf16 with integer operations instead of the conversion unit: together
-// they move work off the special-function pipe, which otherwise bounds the softmax.
-constexpr uint32_t kEmuPairMask = 0x00;
-constexpr uint32_t kIntPackPairMask = 0x00;
+// P is published to the MMA warp in chunks of 64 keys (one mbarrier each, one arrival per
+// softmax warp), so O += P V starts on the first chunk while the softmax still makes the
+// second.  (Smaller chunks add a barrier wait per chunk to the MMA warp, which shares its
+// SM sub-partition with two softmax warps; measured slower.)
+constexpr int kPChunks = 2;
+constexpr int kChunkKeys = kBN / kPChunks;
+
 
 // Operand kinds of the forward: bf16 (kind::f16); FP8: q, k, v in e4m3 (d = 128 only), the
 // S and P V products on the kind::f8f6f4 tensor-core path with P rounded to e4m3; TF32: fp32
@@ -80,7 +87,7 @@ struct FwdCfg {
   static constexpr int kStages = KIND == kKindTF32 ? 4 : ((KIND == kKindFP8 || D == 64) ? 8 : 4);
   static constexpr int kQBytes = 2 * kTileBytes;
   static constexpr int kRingBytes = kStages * kTileBytes;
-  static constexpr int kNumBars = 2 + 2 * kStages + 10;
+  static constexpr int kNumBars = 2 + 2 * kStages + 6 + 2 * kPChunks;
   static constexpr int kBarBytes = kNumBars * 8 + 16;
   static constexpr int kSchedBytes = kMaxVarlenB * 2 + kMaxVarlenT * 4 + 16;
   static constexpr int kSmemBytes = 1024 + kQBytes + kRingBytes + kBarBytes + kSchedBytes;
@@ -177,6 +184,23 @@ struct UnitIter {
   }
 };
 
+// Maximum of 128 scores: 16 independent chains of three-input max, then a three-level tree.
+__device__ __forceinline__ float row_max128(const float (&s)[128]) {
+  float mx[16];
+#pragma unroll
+  for (int q = 0; q < 16; ++q) {
+    mx[q] = fmax3(s[q], s[q + 16], s[q + 32]);
+    mx[q] = fmax3(mx[q], s[q + 48], s[q + 64]);
+    mx[q] = fmax3(mx[q], s[q + 80], s[q + 96]);
+    mx[q] = fmaxf(mx[q], s[q + 112]);
+  }
+  float my[6];
+#pragma unroll
+  for (int q = 0; q < 5; ++q) my[q] = fmax3(mx[3 * q], mx[3 * q + 1], mx[3 * q + 2]);
+  my[5] = mx[15];
+  return fmaxf(fmax3(my[0], my[1], my[2]), fmax3(my[3], my[4], my[5]));
+}
+
 template <int D, bool OUT_F32, int KIND = kKindBF16>
 __global__ void __launch_bounds__(kFwdThreads, 1)
     fa_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
@@ -195,10 +219,10 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
   uint64_t* q_empty = bars + 1;
   uint64_t* full = bars + 2;
   uint64_t* empty = bars + 2 + NS;
-  uint64_t* s_full = bars + 2 + 2 * NS;  // [tile]
-  uint64_t* p_half = s_full + 2;         // [tile][half]: P columns 0-63 / 64-127 written
-  uint64_t* pv_done = p_half + 4;        // [tile]
-  uint64_t* o_free = pv_done + 2;        // [tile]
+  uint64_t* s_full = bars + 2 + 2 * NS;   // [tile]
+  uint64_t* p_chunk = s_full + 2;         // [tile][chunk]: P of keys 32c .. 32c+31 written
+  uint64_t* pv_done = p_chunk + 2 * kPChunks;  // [tile]
+  uint64_t* o_free = pv_done + 2;         // [tile]: O read out by the epilogue
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + C::kNumBars);
   int* sched_misc = reinterpret_cast<int*>(tmem_slot + 2);  // [0] = T, [1] = total tiles
   uint8_t* sched_mem = reinterpret_cast<uint8_t*>(bars) + C::kBarBytes;
@@ -217,10 +241,9 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(s_full + i, 1);
-      mbar_init(p_half + 2 * i, kBM);
-      mbar_init(p_half + 2 * i + 1, kBM);
+      for (int c = 0; c < kPChunks; ++c) mbar_init(p_chunk + kPChunks * i + c, kBM / 32);  // one per warp
       mbar_init(pv_done + i, 1);
-      mbar_init(o_free + i, kBM);
+      mbar_init(o_free + i, kBM / 32);  // one per softmax warp
     }
     sched_misc[0] = 0;
     sched_misc[1] = 0;
@@ -345,48 +368,58 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       UnitWalker wk;
       bool ok = true;
 
-      // k-steps of 32 bytes along d (16 bf16, 32 e4m3 or 8 tf32 elements), four per panel
+      // Shared-memory descriptors are built once; a k-step or a ring slot only moves the
+      // start address (the low 14 bits, in 16-byte units, never carry: shared addresses are
+      // below 2^18 bytes).  The MMAs of one group are issued by one elected lane.
+      const uint64_t dQ = smem_desc_sw128(qbase, 16, 1024);  // K-major, 128-byte swizzle
+      const uint64_t dR = smem_desc_sw128(rbase, 16, 1024);  // ring slots read K-major (K, V^T)
+      const uint64_t dV = smem_desc_sw128(rbase, C::kChunkBytes, 1024);  // bf16 V read MN-major
+      auto slot_off = [](uint32_t slot) -> uint64_t { return (uint64_t)((slot * C::kTileBytes) >> 4); };
+      // S_i = Q_i K^T: k-steps of 32 bytes along d (16 bf16, 32 e4m3 or 8 tf32 elements),
+      // four per 128-byte panel; then commit to the tile's s_full barrier.
       auto issue_S = [&](int i, uint32_t slot) {
+        const uint64_t a0 = dQ + (uint64_t)((i * C::kTileBytes) >> 4), b0 = dR + slot_off(slot);
+        if (elect_one_lane()) {
 #pragma unroll
-        for (int kk = 0; kk < D * C::kElemBytes / 32; ++kk) {
-          const uint32_t off = (kk >> 2) * C::kChunkBytes + (kk & 3) * 32;
-          const uint64_t a = smem_desc_sw128(qbase + i * C::kTileBytes + off, 16, 1024);
-          const uint64_t bd = smem_desc_sw128(rbase + slot * C::kTileBytes + off, 16, 1024);
-          if (FP8)
-            umma_ss_f8_elect(tmem + i * kBN, a, bd, idS, kk > 0 ? 1u : 0u);
-          else if (TF32)
-            umma_ss_tf32_elect(tmem + i * kBN, a, bd, idS, kk > 0 ? 1u : 0u);
-          else
-            umma_ss_elect(tmem + i * kBN, a, bd, idS, kk > 0 ? 1u : 0u);
+          for (int kk = 0; kk < D * C::kElemBytes / 32; ++kk) {
+            const uint32_t off = ((kk >> 2) * C::kChunkBytes + (kk & 3) * 32) >> 4;
+            mma_ss<KIND>(tmem + i * kBN, a0 + off, b0 + off, idS, kk > 0 ? 1u : 0u);
+          }
+          umma_commit(s_full + i);
         }
+        __syncwarp();
       };
-      // O_i (+)= P_i V for the keys of one half (8 k-steps of 16 keys in all).
-      // (P in TMEM: 8 columns per k-step either way, 16 keys of bf16 or 32 keys of e4m3)
-      auto issue_PV_half = [&](int i, uint32_t slot, int half, bool acc) {
-        if (TF32) {
-          // P in fp32 over all 128 columns of S; k-steps of 8 keys (32 bytes of a V^T row)
+      // O_i (+)= P_i V for the 32 keys of chunk c.  P sits in the S columns of its tile:
+      // bf16 two keys per column (k-steps of 16 keys = 8 columns), e4m3 four keys per column
+      // (one k-step of 32 keys = 8 columns), fp32 one key per column (k-steps of 8 keys).
+      auto issue_PV_chunk = [&](int i, uint32_t slot, int c, bool acc) {
+        const uint32_t dO = tmem + C::kColO + i * D, aP = tmem + i * kBN;
+        if (elect_one_lane()) {
+          if constexpr (TF32) {
+            const uint64_t b0 = dR + slot_off(slot);
 #pragma unroll
-          for (int k8 = 0; k8 < kBN / 16; ++k8) {
-            const int kk = half * (kBN / 16) + k8;
-            const uint64_t bd =
-                smem_desc_sw128(rbase + slot * C::kTileBytes + (kk >> 2) * C::kVtPanelBytes + (kk & 3) * 32, 16, 1024);
-            umma_ts_tf32_elect(tmem + C::kColO + i * D, tmem + i * kBN + kk * 8, bd, idPV, (acc || kk > 0) ? 1u : 0u);
-          }
-        } else if (FP8) {
+            for (int k8 = 0; k8 < kChunkKeys / 8; ++k8) {
+              const int kk = c * (kChunkKeys / 8) + k8;  // 8 keys = 32 bytes of each V^T row
+              const uint32_t off = ((kk >> 2) * C::kVtPanelBytes + (kk & 3) * 32) >> 4;
+              mma_ts<KIND>(dO, aP + kk * 8, b0 + off, idPV, (acc || kk > 0) ? 1u : 0u);
+            }
+          } else if constexpr (FP8) {
+            const uint64_t b0 = dR + slot_off(slot);
 #pragma unroll
-          for (int k2 = 0; k2 < kBN / 64; ++k2) {
-            const int kk = half * (kBN / 64) + k2;  // 32 keys = 32 bytes of each V^T row
-            const uint64_t bd = smem_desc_sw128(rbase + slot * C::kTileBytes + kk * 32, 16, 1024);
-            umma_ts_f8_elect(tmem + C::kColO + i * D, tmem + i * kBN + kk * 8, bd, idPV, (acc || kk > 0) ? 1u : 0u);
-          }
-        } else {
+            for (int k32 = 0; k32 < kChunkKeys / 32; ++k32) {
+              const int kk = c * (kChunkKeys / 32) + k32;  // 32 keys = 32 bytes of each V^T row
+              mma_ts<KIND>(dO, aP + kk * 8, b0 + (uint32_t)((kk * 32) >> 4), idPV, (acc || kk > 0) ? 1u : 0u);
+            }
+          } else {
+            const uint64_t b0 = dV + slot_off(slot);
 #pragma unroll
-          for (int k4 = 0; k4 < kBN / 32; ++k4) {
-            const int kk = half * (kBN / 32) + k4;
-            const uint64_t bd = smem_desc_sw128(rbase + slot * C::kTileBytes + kk * 16 * 128, C::kChunkBytes, 1024);
-            umma_ts_elect(tmem + C::kColO + i * D, tmem + i * kBN + kk * 8, bd, idPV, (acc || kk > 0) ? 1u : 0u);
+            for (int k2 = 0; k2 < kChunkKeys / 16; ++k2) {
+              const int kk = c * (kChunkKeys / 16) + k2;  // 16 keys = 16 rows of 128 bytes
+              mma_ts<KIND>(dO, aP + kk * 8, b0 + (uint32_t)((kk * 16 * 128) >> 4), idPV, (acc || kk > 0) ? 1u : 0u);
+            }
           }
         }
+        __syncwarp();
       };
       auto wait_full = [&](uint32_t gi) -> bool {
         if (!warp_wait(full + (gi % NS), (gi / NS) & 1)) return false;
@@ -395,11 +428,11 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       };
       auto pv_step = [&](int i, int j, uint32_t vslot) -> bool {
         if (j == 0 && ounits[i] > 0 && !warp_wait(o_free + i, (ounits[i] - 1) & 1)) return false;
-        // the first half of P is consumed while the softmax still writes the second
-        for (int half = 0; half < 2; ++half) {
-          if (!warp_wait(p_half + 2 * i + half, pcnt[i] & 1)) return false;
+        // each chunk of P is consumed while the softmax still writes the next
+        for (int c = 0; c < kPChunks; ++c) {
+          if (!warp_wait(p_chunk + kPChunks * i + c, pcnt[i] & 1)) return false;
           tc_fence_after();
-          issue_PV_half(i, vslot, half, j > 0);
+          issue_PV_chunk(i, vslot, c, j > 0);
         }
         ++pcnt[i];
         umma_commit_elect(pv_done + i);
@@ -420,12 +453,13 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         // prologue: S_i(0)
         if (!wait_full(g)) break;
         for (int i = 0; i < 2; ++i)
-          if (un.n[i] > 0) {
-            issue_S(i, g % NS);
-            umma_commit_elect(s_full + i);
-          }
+          if (un.n[i] > 0) issue_S(i, g % NS);
         umma_commit_elect(empty + (g % NS));
         if (nmax == 1) umma_commit_elect(q_empty);
+        // per K/V tile j: O_0 += P_0(j) V(j), S_0(j+1), O_1 += P_1(j) V(j), S_1(j+1), so the
+        // tensor core works on one tile while the softmax warps work on the other.  (One
+        // issuing warp per tile lets the tensor core interleave both tiles' products, which
+        // stretches both chains: measured slower.)
         for (int j = 0; j < nmax && ok; ++j) {
           const uint32_t gv = g + 2 * j + 1;
           const uint32_t gk = g + 2 * j + 2;
@@ -433,18 +467,12 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
           if (j < un.n[0] && !pv_step(0, j, gv % NS)) { ok = false; break; }
           if (j + 1 < nmax) {
             if (!wait_full(gk)) { ok = false; break; }
-            if (j + 1 < un.n[0]) {
-              issue_S(0, gk % NS);
-              umma_commit_elect(s_full + 0);
-            }
+            if (j + 1 < un.n[0]) issue_S(0, gk % NS);
           }
           if (j < un.n[1] && !pv_step(1, j, gv % NS)) { ok = false; break; }
           umma_commit_elect(empty + (gv % NS));
           if (j + 1 < nmax) {
-            if (j + 1 < un.n[1]) {
-              issue_S(1, gk % NS);
-              umma_commit_elect(s_full + 1);
-            }
+            if (j + 1 < un.n[1]) issue_S(1, gk % NS);
             umma_commit_elect(empty + (gk % NS));
             if (j + 2 == nmax) umma_commit_elect(q_empty);
           }
@@ -482,6 +510,50 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       const int diag = un.nk - un.nq;                              // causal offset
       float m_ref = -INFINITY, l = 0.f;
 
+      // P of keys 32c .. 32c+31 from the scores s (exponent reference ms, as -ms in both halves
+      // of nms2) into pk, with the row sum of the unrounded values added to lsum.
+      constexpr int kW = FP8 ? kChunkKeys / 4 : (TF32 ? kChunkKeys : kChunkKeys / 2);  // TMEM words
+      const uint64_t tau2 = f2(tau, tau);
+      auto make_chunk = [&](const float (&sc)[128], int c, uint64_t nms2, uint32_t (&pk)[kW], uint64_t (&lsum)[2]) {
+#pragma unroll
+        for (int e = 0; e < kChunkKeys / 2; ++e) {
+          const int g = c * (kChunkKeys / 2) + e;  // column pair
+          float x0, x1;
+          f2_split(f2_fma(f2(sc[2 * g], sc[2 * g + 1]), tau2, nms2), x0, x1);
+          const float p0 = ex2_approx(x0), p1 = ex2_approx(x1);
+          lsum[e & 1] = f2_add(lsum[e & 1], f2(p0, p1));
+          if (TF32) {
+            pk[2 * e] = __float_as_uint(p0);
+            pk[2 * e + 1] = __float_as_uint(p1);
+          } else if (FP8) {
+            // four keys per word: pairs e (even) and e + 1 share one
+            if (e & 1) pk[e >> 1] |= pack_e4m3x2_hi(p0, p1);
+            else pk[e >> 1] = pack_e4m3x2_lo(p0, p1);
+          } else {
+            pk[e] = pack_bf16x2(p0, p1);
+          }
+        }
+      };
+      // Writes chunk c of P over the S columns of its tile and tells the MMA warp (one arrival
+      // per warp, after every lane's store has completed).
+      auto publish = [&](int c, const uint32_t (&pk)[kW]) {
+        const uint32_t col = (uint32_t)(c * kW);
+        if constexpr (kW == 64) {
+          tmem_st32(tS + col, reinterpret_cast<const uint32_t(&)[32]>(pk[0]));
+          tmem_st32(tS + col + 32, reinterpret_cast<const uint32_t(&)[32]>(pk[32]));
+        } else if constexpr (kW == 32) {
+          tmem_st32(tS + col, pk);
+        } else if constexpr (kW == 16) {
+          tmem_st16(tS + col, pk);
+        } else {
+          tmem_st8(tS + col, pk);
+        }
+        tmem_wait_st();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(p_chunk + kPChunks * i + c);
+      };
+
       for (int j = 0; j < n; ++j) {
         if (!mbar_wait(s_full + i, scnt & 1)) { ok = false; break; }
         ++scnt;
@@ -496,6 +568,36 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
 
         const int key0 = j * kBN;
         const bool need_mask = (key0 + kBN > un.nk) || (p.causal && key0 + kBN - 1 > warp_row_min + diag);
+        uint64_t lsum[2] = {f2(0.f, 0.f), f2(0.f, 0.f)};
+        float m_tile;
+        bool have_max = false;
+        // Speculative step: once every row of the warp has a finite reference max and no key
+        // of this tile is masked, exponentiate against the reference at once.  The tile max,
+        // computed alongside the first chunk's exponentials, then only has to confirm that no
+        // row rose above the lazy threshold before anything is published; if one did, the
+        // chunk is dropped and the full step below runs (the exact result is the same either
+        // way: O and l always share the reference).
+        if (!need_mask && __all_sync(0xffffffffu, m_ref != -INFINITY)) {
+          m_tile = row_max128(s) * tau;
+          const uint64_t nms2 = f2(-m_ref, -m_ref);
+          uint32_t pk[kW];
+          make_chunk(s, 0, nms2, pk, lsum);
+          if (!__any_sync(0xffffffffu, m_tile - m_ref > kRescaleThreshold)) {
+            publish(0, pk);
+#pragma unroll
+            for (int c = 1; c < kPChunks; ++c) {
+              make_chunk(s, c, nms2, pk, lsum);
+              publish(c, pk);
+            }
+            float la, lb, lc, ld;
+            f2_split(lsum[0], la, lb);
+            f2_split(lsum[1], lc, ld);
+            l += (la + lb) + (lc + ld);
+            continue;
+          }
+          lsum[0] = lsum[1] = f2(0.f, 0.f);
+          have_max = true;
+        }
         if (need_mask) {
           int lim = un.nk - key0;
           if (p.causal) lim = min(lim, row + diag + 1 - key0);
@@ -503,20 +605,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
           for (int c = 0; c < 128; ++c)
             if (c >= lim) s[c] = -INFINITY;
         }
-        // row max: 16 independent chains of three-input max, then a three-level tree
-        float mx[16];
-#pragma unroll
-        for (int q = 0; q < 16; ++q) {
-          mx[q] = fmax3(s[q], s[q + 16], s[q + 32]);
-          mx[q] = fmax3(mx[q], s[q + 48], s[q + 64]);
-          mx[q] = fmax3(mx[q], s[q + 80], s[q + 96]);
-          mx[q] = fmaxf(mx[q], s[q + 112]);
-        }
-        float my[6];
-#pragma unroll
-        for (int q = 0; q < 5; ++q) my[q] = fmax3(mx[3 * q], mx[3 * q + 1], mx[3 * q + 2]);
-        my[5] = mx[15];
-        const float m_tile = fmaxf(fmax3(my[0], my[1], my[2]), fmax3(my[3], my[4], my[5])) * tau;
+        if (!have_max) m_tile = row_max128(s) * tau;
         const float m_new = fmaxf(m_ref, m_tile);
         const bool need = m_new - m_ref > kRescaleThreshold;  // false when both are -inf
         const bool warp_need = __any_sync(0xffffffffu, need);
@@ -539,64 +628,14 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
           }
           tmem_wait_st();
         }
-        // P = 2^(t - m_ref) as packed bf16 over the first 64 columns of S, published in two
-        // halves of 64 keys so the P V product starts on the first while the second is made.
+        // P = 2^(t - m_ref), chunk by chunk, each published as soon as it is written
         const float ms = (m_ref == -INFINITY) ? 0.f : m_ref;
-        const uint64_t tau2 = f2(tau, tau), nms2 = f2(-ms, -ms);
-        uint64_t lsum[2] = {f2(0.f, 0.f), f2(0.f, 0.f)};
+        const uint64_t nms2 = f2(-ms, -ms);
 #pragma unroll
-        for (int half = 0; half < 2; ++half) {
-          if (TF32) {
-            // fp32 P over the S columns of its own keys (read by the tensor core as tf32)
-            uint32_t pk[2][32];
-#pragma unroll
-            for (int e = 0; e < 32; ++e) {
-              const int g = 32 * half + e;  // column pair
-              float x0, x1;
-              f2_split(f2_fma(f2(s[2 * g], s[2 * g + 1]), tau2, nms2), x0, x1);
-              const float p0 = ex2_approx(x0), p1 = ex2_approx(x1);
-              lsum[g & 1] = f2_add(lsum[g & 1], f2(p0, p1));
-              pk[e >> 4][2 * (e & 15)] = __float_as_uint(p0);
-              pk[e >> 4][2 * (e & 15) + 1] = __float_as_uint(p1);
-            }
-            tmem_st32(tS + 64 * half, pk[0]);
-            tmem_st32(tS + 64 * half + 32, pk[1]);
-          } else if (FP8) {
-            // e4m3 P, four keys per TMEM column: 64 keys in 16 columns
-            uint32_t pk[16];
-#pragma unroll
-            for (int e = 0; e < 16; ++e) {
-              const int g = 32 * half + 2 * e;  // first of two column pairs
-              float x0, x1, x2, x3;
-              f2_split(f2_fma(f2(s[2 * g], s[2 * g + 1]), tau2, nms2), x0, x1);
-              f2_split(f2_fma(f2(s[2 * g + 2], s[2 * g + 3]), tau2, nms2), x2, x3);
-              const float p0 = ex2_approx(x0), p1 = ex2_approx(x1), p2 = ex2_approx(x2), p3 = ex2_approx(x3);
-              lsum[0] = f2_add(lsum[0], f2(p0, p1));
-              lsum[1] = f2_add(lsum[1], f2(p2, p3));
-              pk[e] = pack_e4m3x4(p0, p1, p2, p3);
-            }
-            tmem_st16(tS + 16 * half, pk);
-          } else {
-            uint32_t pk[32];
-#pragma unroll
-            for (int e = 0; e < 32; ++e) {
-              const int g = 32 * half + e;  // column pair
-              float x0, x1, p0, p1;
-              f2_split(f2_fma(f2(s[2 * g], s[2 * g + 1]), tau2, nms2), x0, x1);
-              if (((kEmuPairMask >> (g & 7)) & 1u) && !need_mask) {
-                exp2_poly_x2(x0, x1, p0, p1);
-              } else {
-                p0 = ex2_approx(x0);
-                p1 = ex2_approx(x1);
-              }
-              lsum[g & 1] = f2_add(lsum[g & 1], f2(p0, p1));
-              pk[e] = ((kIntPackPairMask >> (g & 7)) & 1u) ? pack_bf16x2_int(p0, p1) : pack_bf16x2(p0, p1);
-            }
-            tmem_st32(tS + 32 * half, pk);
-          }
-          tmem_wait_st();
-          tc_fence_before();
-          mbar_arrive(p_half + 2 * i + half);
+        for (int c = 0; c < kPChunks; ++c) {
+          uint32_t pk[kW];
+          make_chunk(s, c, nms2, pk, lsum);
+          publish(c, pk);
         }
         float la, lb, lc, ld;
         f2_split(lsum[0], la, lb);
@@ -605,7 +644,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       }
       if (!ok) break;
 
-      // ---- epilogue: O / l, lse
+      // ---- epilogue: O / l (times the output scale) -> HBM, lse = (m + log2 l) ln 2
       if (n > 0) {
         if (!mbar_wait(pv_done + i, (pvcnt + n - 1) & 1)) { ok = false; break; }
         tc_fence_after();
@@ -623,6 +662,12 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         } else {
 #pragma unroll
           for (int e = 0; e < 32; ++e) ov[e] = 0u;
+        }
+        if (c == D / 32 - 1 && n > 0) {
+          // every column of O is in registers: the next unit's products may overwrite it
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(o_free + i);
         }
         if (row_ok) {
           if (OUT_F32) {
@@ -650,10 +695,6 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         const size_t li = (p.cu != nullptr) ? (size_t)un.h * p.Nq + un.q_start + row
                                              : ((size_t)un.b * p.Hq + un.h) * p.Nq + row;
         p.lse[li] = v;
-      }
-      if (n > 0) {
-        tc_fence_before();
-        mbar_arrive(o_free + i);
       }
     }
   }

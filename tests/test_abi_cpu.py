@@ -213,6 +213,57 @@ def test_binding_checks_index_types_and_output_shapes(lib):
                         torch.zeros(2, dtype=torch.int32), stream=0)
 
 
+def test_binding_checks_shapes_across_tensors(lib):
+    """The kernels size every read from q's batch, heads and head dimension: a k, cache or
+    length vector that does not match q is refused by the binding with a ValueError (a
+    smaller tensor would otherwise be read past its end on the device)."""
+    import torch
+    bf, i32 = torch.bfloat16, torch.int32
+    q = torch.zeros(2, 16, 4, 64, dtype=bf)
+    with pytest.raises(ValueError, match="batch 2"):
+        fa.forward(q, torch.zeros(1, 16, 2, 64, dtype=bf), torch.zeros(1, 16, 2, 64, dtype=bf), stream=0)
+    with pytest.raises(ValueError, match="multiple of Hkv"):
+        fa.forward(q, torch.zeros(2, 16, 3, 64, dtype=bf), torch.zeros(2, 16, 3, 64, dtype=bf), stream=0)
+    qp = torch.zeros(40, 4, 64, dtype=bf)
+    with pytest.raises(ValueError, match="packed rows"):
+        fa.forward(qp, torch.zeros(39, 2, 64, dtype=bf), torch.zeros(39, 2, 64, dtype=bf),
+                   cu_seqlens=torch.tensor([0, 40], dtype=i32), stream=0)
+    with pytest.raises(ValueError, match="cu_seqlens"):
+        fa.forward(qp, torch.zeros(40, 2, 64, dtype=bf), torch.zeros(40, 2, 64, dtype=bf),
+                   cu_seqlens=torch.tensor([40], dtype=i32), stream=0)
+    qd = torch.zeros(2, 8, 128, dtype=bf)
+    with pytest.raises(ValueError, match="kcache"):   # cache of one sequence for two queries
+        fa.decode(qd, torch.zeros(1, 64, 2, 128, dtype=bf), torch.zeros(1, 64, 2, 128, dtype=bf), stream=0)
+    with pytest.raises(ValueError, match="kcache"):   # head dimension differs from q's
+        fa.decode(qd, torch.zeros(2, 64, 2, 64, dtype=bf), torch.zeros(2, 64, 2, 64, dtype=bf), stream=0)
+    with pytest.raises(ValueError, match="seqlens"):
+        fa.decode(qd, torch.zeros(2, 64, 2, 128, dtype=bf), torch.zeros(2, 64, 2, 128, dtype=bf),
+                  seqlens=torch.zeros(1, dtype=i32), stream=0)
+    with pytest.raises(ValueError, match="multiple of Hkv"):
+        fa.decode(qd, torch.zeros(2, 64, 3, 128, dtype=bf), torch.zeros(2, 64, 3, 128, dtype=bf), stream=0)
+    with pytest.raises(ValueError, match="k_pages"):
+        fa.decode_paged(qd, torch.zeros(8, 16, 2, 64, dtype=bf), torch.zeros(8, 16, 2, 64, dtype=bf),
+                        torch.zeros(2, 4, dtype=i32), torch.zeros(2, dtype=i32), stream=0)
+    with pytest.raises(ValueError, match="seqlens"):
+        fa.decode_paged(qd, torch.zeros(8, 16, 2, 128, dtype=bf), torch.zeros(8, 16, 2, 128, dtype=bf),
+                        torch.zeros(2, 4, dtype=i32), torch.zeros(3, dtype=i32), stream=0)
+    lse = torch.zeros(2, 4, 16, dtype=torch.float32)
+    with pytest.raises(ValueError, match="k"):
+        fa.backward(q, torch.zeros(1, 16, 2, 64, dtype=bf), torch.zeros(1, 16, 2, 64, dtype=bf), q, lse, q, stream=0)
+    with pytest.raises(ValueError, match="d=64"):
+        fa.backward(q, torch.zeros(2, 16, 2, 128, dtype=bf), torch.zeros(2, 16, 2, 128, dtype=bf), q, lse, q,
+                    stream=0)
+    with pytest.raises(ValueError, match="total=40"):
+        fa.backward_varlen(qp, torch.zeros(39, 2, 64, dtype=bf), torch.zeros(39, 2, 64, dtype=bf), qp,
+                           torch.zeros(4, 40), qp, torch.tensor([0, 40], dtype=i32), stream=0)
+    with pytest.raises(ValueError, match="qkv"):
+        fa.forward_qkvpacked(torch.zeros(2, 16, 2, 4, 64, dtype=bf))
+    u8 = torch.uint8
+    with pytest.raises(ValueError, match="k8"):
+        fa.forward_fp8(torch.zeros(2, 16, 4, 128, dtype=u8), torch.zeros(1, 16, 2, 128, dtype=u8),
+                       torch.zeros(1, 16, 2, 128, dtype=u8), 1.0, 1.0, 1.0)
+
+
 def test_bwd_rejects_before_launch(lib):
     def st(**kw):
         a = dict(q=256, k=256, v=256, o=256, do=256, lse=512, dq=256, dk=256, dv=256, B=1, Hq=2, Hkv=1, Nq=8, Nk=8,
