@@ -5,8 +5,9 @@ workload (B=1, Hq=64, Hkv=8, N=8192, d=128, bf16) and the split-KV decode on the
 workload (B=8, Hq=64, Hkv=8, cache 32768, d=128, splits of 1024).  The headline value is the
 forward's TFLOP/s (4 B Hq N^2 d, halved for causal); the decode's HBM GB/s (K and V bytes
 read once) is reported in the "decode" object.  Inputs are synthetic i.i.d. N(0,1) from the
-seeded generator, resident in HBM before timing; L2 is flushed (a 256 MiB write) before every
-timed launch, outside its events.
+seeded generator, resident in HBM before timing; L2 is flushed before every timed launch,
+outside its events: a 256 MiB write, then a read of another 256 MiB buffer, so that the
+write's dirty lines are written back before the launch rather than during it.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
 
@@ -231,9 +232,13 @@ def run_device(args):
         torch.cuda.synchronize()
 
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    flush_rd = torch.ones(64 << 20, dtype=torch.float32, device=dev)  # 256 MiB
 
     def l2_flush():
+        # write a buffer larger than L2, then read another one: L2 holds neither the previous
+        # launch's data nor dirty lines whose write-back would land inside the timed launch
         flush.fill_(1)
+        flush_rd.sum()
 
     # ---- inputs (each rank its own replica, seeded by the workload seed + rank)
     w = FWD
@@ -256,6 +261,8 @@ def run_device(args):
     do_fp8 = args.only in ("all", "fp8")
     do_tf32 = args.only in ("all", "tf32")
     do_bwdv = args.only == "bwd_varlen"  # on request only: its inputs take about a minute to draw
+    do_mha2k = args.only in ("all", "mha2k")
+    do_varlen = args.only in ("all", "varlen")
     if do_bwd:
         h_do_f = torch.from_numpy(inputs("fwd", seed, DOUT_ID, (B, N, Hq, d))).to(torch.bfloat16)
         b_do = h_do_f.to(dev)
@@ -337,6 +344,35 @@ def run_device(args):
         v_ws_bytes = fa.fa_bwd_varlen_workspace_size(vB, vHq, vT, vd)
         v_ws = torch.empty(v_ws_bytes, dtype=torch.uint8, device=dev)
 
+    if do_mha2k:
+        wm = MHA2K
+        mB, mN, mH, md = wm["B"], wm["N"], wm["Hq"], wm["d"]
+        mseed = replica_seed(wm["seed"], rank)
+        m_q, m_k, m_v = (torch.from_numpy(inputs("mha2k", mseed, tid, (mB, mN, mH, md))).to(torch.bfloat16).to(dev)
+                         for tid in (si.Q, si.K, si.V))
+        m_o = torch.empty_like(m_q)
+        m_lse = torch.empty((mB, mH, mN), dtype=torch.float32, device=dev)
+
+    if do_varlen:
+        fseed = replica_seed(VARLEN["seed"], rank)
+        f_len = varlen_lengths(VARLEN["seed"])  # the same lengths on every rank, own values
+        f_cu_np = si.cu_seqlens(f_len)
+        fT, fB = int(f_cu_np[-1]), len(f_len)
+        fHq, fHkv, fd = VARLEN["Hq"], VARLEN["Hkv"], VARLEN["d"]
+        f_q, f_k, f_v = (torch.from_numpy(inputs("varlen", fseed, tid, (fT, hh, fd))).to(torch.bfloat16).to(dev)
+                         for tid, hh in ((si.Q, fHq), (si.K, fHkv), (si.V, fHkv)))
+        f_cu = torch.from_numpy(f_cu_np).to(dev)
+        f_o = torch.empty_like(f_q)
+        f_lse = torch.empty((fHq, fT), dtype=torch.float32, device=dev)
+
+    def call_mha2k():
+        fa.fa_fwd(m_q, m_k, m_v, m_o, m_lse, mB, mH, mH, mN, mN, md, 1.0 / math.sqrt(md), 1, None, fa.FA_BF16, None, 0,
+                  st)
+
+    def call_varlen():
+        fa.fa_fwd(f_q, f_k, f_v, f_o, f_lse, fB, fHq, fHkv, fT, fT, fd, 1.0 / math.sqrt(fd), 1, f_cu, fa.FA_BF16,
+                  None, 0, st)
+
     def call_bwdv():
         fa.fa_bwd_varlen(v_q, v_k, v_v, v_o, v_do, v_lse, v_dq, v_dk, v_dv, vB, vHq, vHkv, vT, vd, vscale, 1, v_cu,
                          v_ws, v_ws_bytes, st)
@@ -393,6 +429,8 @@ def run_device(args):
     fp8_ms = timed_launches(call_fp8, args.steps, args.warmup) if do_fp8 else [float("nan")]
     tf32_ms = timed_launches(call_tf32, args.steps, args.warmup) if do_tf32 else [float("nan")]
     bwdv_ms = timed_launches(call_bwdv, args.steps, args.warmup) if do_bwdv else [float("nan")]
+    mha2k_ms = timed_launches(call_mha2k, args.steps, args.warmup) if do_mha2k else [float("nan")]
+    varlen_ms = timed_launches(call_varlen, args.steps, args.warmup) if do_varlen else [float("nan")]
     if fa.fa_last_device_error(st) != fa.FA_OK:
         raise RuntimeError("device-side timeout recorded during the benchmark")
 
@@ -440,6 +478,8 @@ def run_device(args):
     fp8_mean = max_over_ranks(sum(fp8_ms) / len(fp8_ms), dev)
     tf32_mean = max_over_ranks(sum(tf32_ms) / len(tf32_ms), dev)
     bwdv_mean = max_over_ranks(sum(bwdv_ms) / len(bwdv_ms), dev)
+    mha2k_mean = max_over_ranks(sum(mha2k_ms) / len(mha2k_ms), dev)
+    varlen_mean = max_over_ranks(sum(varlen_ms) / len(varlen_ms), dev)
     fwd_e2e_ms = max_over_ranks(fwd_e2e_ms, dev)
     dec_e2e_ms = max_over_ranks(dec_e2e_ms, dev)
     if world > 1:
@@ -488,7 +528,8 @@ def run_device(args):
         "config": {"workload": "gqa_causal_8k: B=1, Hq=64, Hkv=8, N=8192, d=128, causal, layout [B,N,H,d]",
                    "decode_workload": "decode_split_kv: B=8, Hq=64, Hkv=8, cache 32768, d=128, split 1024",
                    "parallelism": f"replicas x{world} (independent units, no collective)",
-                   "l2": "flushed before every timed launch (256 MiB write, outside the events)",
+                   "l2": "flushed before every timed launch, outside the events (256 MiB write, then a 256 MiB read of "
+                              "another buffer so the write-back happens before the launch)",
                    "timing": "CUDA events around each launch on the launching stream; mean over steps; max over ranks"},
         "roofline": {"bound": "tensor", "achieved": round(per_launch_tflops, 2), "peak": tc_peak, "unit": "TFLOP/s",
                      "frac": round(per_launch_tflops / tc_peak, 4),
@@ -550,11 +591,43 @@ def run_device(args):
                 "h2d_bytes_per_step": h2d_fwd, "d2h_bytes_per_step": d2h_fwd},
         "cpu_baseline": cpu,
         "gpu_launches": args.steps * (int(do_fwd) * 1 + int(do_dec) * 2 + int(do_paged) * 1 + int(do_bwd) * 3 + int(do_fp8) * 2 + int(do_tf32) * 4
-                                     + int(do_bwdv) * 4)
+                                     + int(do_bwdv) * 4 + int(do_mha2k) + int(do_varlen))
         + (0 if args.no_e2e else e2e_steps * (int(do_fwd) * 1 + int(do_dec) * 2)),
         "clocks": clocks.summary(),
         "impl": "b200",
     }
+    if do_mha2k:
+        mF = fwd_flops(MHA2K)
+        m_tflops = mF / (mha2k_mean * 1e-3) / 1e12
+        m_peak = peaks["bf16"] if (args.steps * mha2k_mean) < 1000.0 else peaks["bf16_sustained"]
+        line["forward_mha2k"] = {
+            "value": round(aggregate_rate(mF, world, mha2k_mean) / 1e12, 2), "unit": "TFLOP/s",
+            "ms": round(mha2k_mean, 4),
+            "workload": "mha_causal_2k: B=2, H=12, N=2048, d=64, causal, bf16, layout [B,N,H,d] "
+                        "(latency-sized: 384 query tiles for 148 SMs; reported, no target)",
+            "roofline": {"bound": "tensor", "achieved": round(m_tflops, 2), "peak": m_peak, "unit": "TFLOP/s",
+                         "frac": round(m_tflops / m_peak, 4), "peak_kind": f"measured ({peaks['source']})",
+                         "frac_of_spec_2250": round(m_tflops / SPEC_BF16_TFLOPS, 4),
+                         "traffic": ncu_traffic("fa_fwd/mha_causal_2k"),
+                         "kernel": "fa_fwd_kernel<64,false>", "algorithmic_flops_per_launch": mF,
+                         "algorithmic_bytes_per_launch": fwd_bytes(MHA2K)}}
+    if do_varlen:
+        fF = varlen_flops(f_len)
+        fbytes = float(fT) * (2.0 * 2 * fHq * fd + 2.0 * 2 * fHkv * fd + 4.0 * fHq)
+        f_tflops = fF / (varlen_mean * 1e-3) / 1e12
+        f_peak = peaks["bf16"] if (args.steps * varlen_mean) < 1000.0 else peaks["bf16_sustained"]
+        line["forward_varlen"] = {
+            "value": round(aggregate_rate(fF, world, varlen_mean) / 1e12, 2), "unit": "TFLOP/s",
+            "ms": round(varlen_mean, 4),
+            "workload": f"varlen_gqa_causal: {fB} packed sequences, lengths U[256, 8192] (seed {VARLEN['seed']}), "
+                        f"{fT} rows, Hq=32, Hkv=8, d=128, causal within each sequence",
+            "flops_convention": "sum over sequences of 4 Hq L^2 d / 2",
+            "roofline": {"bound": "tensor", "achieved": round(f_tflops, 2), "peak": f_peak, "unit": "TFLOP/s",
+                         "frac": round(f_tflops / f_peak, 4), "peak_kind": f"measured ({peaks['source']})",
+                         "frac_of_spec_2250": round(f_tflops / SPEC_BF16_TFLOPS, 4),
+                         "traffic": ncu_traffic("fa_fwd/varlen_gqa_causal"),
+                         "kernel": "fa_fwd_kernel<128,false> (varlen schedule)",
+                         "algorithmic_flops_per_launch": fF, "algorithmic_bytes_per_launch": fbytes}}
     if do_bwdv:
         vF = 2.5 * varlen_flops(v_len)
         v_tflops = vF / (bwdv_mean * 1e-3) / 1e12
@@ -697,7 +770,8 @@ def main():
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--no-cpu", action="store_true", help="skip the CPU oracle baseline")
     ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer end-to-end phases")
-    ap.add_argument("--only", default="all", choices=["all", "fwd", "dec", "paged", "bwd", "fp8", "tf32", "bwd_varlen"],
+    ap.add_argument("--only", default="all", choices=["all", "fwd", "dec", "paged", "bwd", "fp8", "tf32", "bwd_varlen",
+                                                       "mha2k", "varlen"],
                     help="profiling: run one kernel family")
     args = ap.parse_args()
     if args.warmup < 3:

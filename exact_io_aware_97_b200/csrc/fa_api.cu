@@ -89,6 +89,10 @@ __global__ void __launch_bounds__(256) transpose_v_f32_kernel(const float* __res
   }
 }
 
+// Reads and clears the error word in one atomic step, so that a record made by a kernel on
+// another stream between a read and a separate clear cannot be lost.
+__global__ void take_error_word_kernel() { g_error_taken = atomicExch(&g_error_word, 0u); }
+
 namespace {
 
 using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
@@ -300,9 +304,11 @@ size_t fa_fwd_workspace_size(int B, int Hq, int Hkv, int Nq, int Nk, int d, fa_d
     return align_up((size_t)B * Nq * Hq * d * 4, 256) + align_up((size_t)B * Nk * Hkv * d * 4, 256) +
            align_up((size_t)B * Hkv * d * pad * 4, 256);
   }
-  if (in_dtype != FA_F32 || varlen) return 0;
+  if (in_dtype != FA_F32) return 0;
   if (B <= 0 || Hq <= 0 || Hkv <= 0 || Nq < 0 || Nk < 0 || d <= 0) return 0;
-  const size_t nq = (size_t)B * Nq * Hq * d, nk = (size_t)B * Nk * Hkv * d;
+  // bf16 copies of q, k, v (varlen: Nq = Nk = the packed row count)
+  const size_t rq = varlen ? (size_t)Nq : (size_t)B * Nq, rk = varlen ? (size_t)Nk : (size_t)B * Nk;
+  const size_t nq = rq * Hq * d, nk = rk * Hkv * d;
   return align_up(nq * 2, 256) + 2 * align_up(nk * 2, 256);
 }
 
@@ -390,7 +396,6 @@ fa_status fa_fwd(const void* q, const void* k, const void* v, void* o, float* ls
   const bool varlen = cu_seqlens != nullptr;
   if (varlen) {
     if (Nq != Nk) return FA_ERR_INVALID_ARG;
-    if (in_dtype != FA_BF16) return FA_ERR_UNSUPPORTED;
     if (B > kMaxVarlenB || (int64_t)Nq > (int64_t)kMaxVarlenT * kUnitRows) return FA_ERR_UNSUPPORTED;
     if ((reinterpret_cast<uintptr_t>(cu_seqlens) & 3u) != 0) return FA_ERR_INVALID_ARG;
   }
@@ -404,7 +409,7 @@ fa_status fa_fwd(const void* q, const void* k, const void* v, void* o, float* ls
                                            workspace_bytes, st);
   const void *qb = q, *kb = k, *vb = v;
   if (in_dtype == FA_F32) {
-    const size_t need = fa_fwd_workspace_size(B, Hq, Hkv, Nq, Nk, d, in_dtype, 0);
+    const size_t need = fa_fwd_workspace_size(B, Hq, Hkv, Nq, Nk, d, in_dtype, varlen ? 1 : 0);
     if (!workspace || workspace_bytes < need || !aligned16(workspace)) return FA_ERR_WORKSPACE;
     const size_t nq = (size_t)rows_q * Hq * d, nk = (size_t)rows_k * Hkv * d;
     uint8_t* w = static_cast<uint8_t*>(workspace);
@@ -783,16 +788,17 @@ fa_status fa_bwd_varlen(const void* q, const void* k, const void* v, const void*
 
 fa_status fa_last_device_error(void* stream) {
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  // one host thread at a time uses g_error_taken
+  static std::mutex mu;
+  std::lock_guard<std::mutex> lock(mu);
+  take_error_word_kernel<<<1, 1, 0, st>>>();
+  if (cudaGetLastError() != cudaSuccess) return FA_ERR_CUDA;
   if (cudaStreamSynchronize(st) != cudaSuccess) return FA_ERR_CUDA;
   unsigned int w = 0;
-  if (cudaMemcpyFromSymbol(&w, g_error_word, sizeof(w)) != cudaSuccess) return FA_ERR_CUDA;
-  if (w != 0) {
-    const unsigned int zero = 0;
-    if (cudaMemcpyToSymbol(g_error_word, &zero, sizeof(zero)) != cudaSuccess) return FA_ERR_CUDA;
-    if (w & kErrTimeout) return FA_ERR_TIMEOUT;
-    if (w & kErrSmem) return FA_ERR_CUDA;
-    return FA_ERR_INVALID_ARG;
-  }
+  if (cudaMemcpyFromSymbol(&w, g_error_taken, sizeof(w)) != cudaSuccess) return FA_ERR_CUDA;
+  if (w & kErrTimeout) return FA_ERR_TIMEOUT;
+  if (w & kErrSmem) return FA_ERR_CUDA;
+  if (w != 0) return FA_ERR_INVALID_ARG;
   return FA_OK;
 }
 

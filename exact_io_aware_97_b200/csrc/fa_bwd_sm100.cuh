@@ -68,8 +68,6 @@ struct BwdParams {
 
 constexpr int kBwdThreads = 384;
 constexpr int kBwdTile = 128;            // keys per CTA tile and queries per pair
-constexpr unsigned int kErrSmem = 4u;    // the kernel's shared-memory carve did not fit
-constexpr unsigned int kErrBadSeqlens = 8u;  // cu_seqlens not non-decreasing within [0, total]
 constexpr int kBwdMaxSmem = 232448;      // sm_100 per-block limit
 
 template <int D>

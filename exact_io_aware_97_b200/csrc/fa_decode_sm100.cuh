@@ -44,7 +44,6 @@ struct DecParams {
   float tau;
 };
 
-constexpr unsigned int kErrBadPage = 2u;  // a block-table entry outside [0, num_pages)
 
 constexpr int kDecKeys = 64;  // cache rows per stage
 constexpr int kDecComputeWarps = 4;

@@ -9,10 +9,16 @@
 
 namespace fa {
 
-// Recorded by any wait that exceeded its time limit; read and cleared by the host.
+// Recorded by any wait that exceeded its time limit and by the device-side input checks;
+// taken (read and cleared in one atomic exchange) by fa_last_device_error.
 __device__ unsigned int g_error_word;
+__device__ unsigned int g_error_taken;  // where that exchange leaves the value for the host
 
-constexpr unsigned int kErrTimeout = 1u;
+// Bits of the error word (fa_last_device_error maps them to a status and clears them).
+constexpr unsigned int kErrTimeout = 1u;       // a bounded wait ran out
+constexpr unsigned int kErrBadPage = 2u;       // a block-table entry outside [0, num_pages)
+constexpr unsigned int kErrSmem = 4u;          // a kernel's shared-memory carve did not fit
+constexpr unsigned int kErrBadSeqlens = 8u;    // cu_seqlens not non-decreasing within [0, total]
 // A wait gives up after this many nanoseconds of %globaltimer (a correct kernel waits
 // microseconds at most); it then records kErrTimeout and reports failure to its caller.
 constexpr unsigned long long kWaitLimitNs = 4000000000ull;
@@ -76,18 +82,17 @@ __device__ __forceinline__ bool mbar_test(uint64_t* bar, uint32_t parity) {
 }
 
 // Waits until the phase with the given parity has completed.  Returns false (and records
-// kErrTimeout) if that takes longer than kWaitLimitNs; the caller then stops its role.
+// kErrTimeout) if that takes longer than kWaitLimitNs; the caller then stops its role.  Each
+// wait times out on its own clock: a timeout recorded by another kernel (or by this one
+// earlier) does not cut later waits short, so one failure never aborts unrelated launches.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
   if (mbar_try_wait(bar, parity)) return true;
   const unsigned long long t0 = globaltimer_ns();
   for (uint32_t it = 0;; ++it) {
     if (mbar_try_wait(bar, parity)) return true;
-    if ((it & 255u) == 255u) {
-      if (globaltimer_ns() - t0 > kWaitLimitNs) {
-        atomicOr(&g_error_word, kErrTimeout);
-        return false;
-      }
-      if (*reinterpret_cast<volatile unsigned int*>(&g_error_word) & kErrTimeout) return false;
+    if ((it & 255u) == 255u && globaltimer_ns() - t0 > kWaitLimitNs) {
+      atomicOr(&g_error_word, kErrTimeout);
+      return false;
     }
   }
 }
@@ -499,6 +504,11 @@ __device__ __forceinline__ void f2_split(uint64_t v, float& a, float& b) {
 __device__ __forceinline__ uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c) {
   uint64_t d;
   asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+__device__ __forceinline__ uint64_t f2_mul(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
   return d;
 }
 __device__ __forceinline__ uint64_t f2_add(uint64_t a, uint64_t b) {

@@ -269,11 +269,21 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
     __syncthreads();
   } else {
     __syncthreads();  // sched_misc initialised
+    // cu_seqlens must start at or above 0, never decrease and end at or below the packed row
+    // count; otherwise no unit is scheduled (nothing is read or written) and the error word
+    // records it for fa_last_device_error.
+    int bad = 0;
     for (int b = threadIdx.x; b < p.B; b += blockDim.x) {
-      const int len = __ldg(p.cu + b + 1) - __ldg(p.cu + b);
+      const int c0 = __ldg(p.cu + b), c1 = __ldg(p.cu + b + 1);
+      bad |= (c1 < c0) | (b == 0 && c0 < 0) | (b == p.B - 1 && c1 > p.Nq);
+      const int len = c1 - c0;
       const int nt = len > 0 ? (len + kUnitRows - 1) / kUnitRows : 0;
       atomicMax(&sched_misc[0], nt);
       atomicAdd(&sched_misc[1], nt);
+    }
+    if (__syncthreads_or(bad)) {
+      if (threadIdx.x == 0) atomicOr(&g_error_word, kErrBadSeqlens);
+      sched_misc[1] = 0;  // (every thread writes the same value)
     }
     __syncthreads();
     const int T = min(sched_misc[0], kMaxVarlenT);
@@ -538,11 +548,10 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       // per warp, after every lane's store has completed).
       auto publish = [&](int c, const uint32_t (&pk)[kW]) {
         const uint32_t col = (uint32_t)(c * kW);
-        if constexpr (kW == 64) {
-          tmem_st32(tS + col, reinterpret_cast<const uint32_t(&)[32]>(pk[0]));
-          tmem_st32(tS + col + 32, reinterpret_cast<const uint32_t(&)[32]>(pk[32]));
-        } else if constexpr (kW == 32) {
-          tmem_st32(tS + col, pk);
+        if constexpr (kW >= 32) {
+#pragma unroll
+          for (int w0 = 0; w0 < kW; w0 += 32)
+            tmem_st32(tS + col + w0, reinterpret_cast<const uint32_t(&)[32]>(pk[w0]));
         } else if constexpr (kW == 16) {
           tmem_st16(tS + col, pk);
         } else {

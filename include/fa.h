@@ -63,14 +63,17 @@ typedef enum { FA_BF16 = 0, FA_F32 = 1, FA_TF32 = 2 } fa_dtype;
  *
  * Fixed length (cu_seqlens == NULL):
  *   q [B, Nq, Hq, d], k and v [B, Nk, Hkv, d], o [B, Nq, Hq, d], lse [B, Hq, Nq].
- * Variable length (cu_seqlens != NULL, device int32 [B+1], cu_seqlens[0] = 0, non-decreasing):
+ * Variable length (cu_seqlens != NULL, device int32 [B+1]):
  *   Nq == Nk == total packed rows; q and o [total, Hq, d], k and v [total, Hkv, d],
  *   lse [Hq, total]; sequence b owns rows [cu_seqlens[b], cu_seqlens[b+1]) of q, k and v and
- *   attends only within itself.  The caller guarantees cu_seqlens[B] <= total (it is read
- *   on the device only).  B <= 1024.
+ *   attends only within itself.  cu_seqlens must start at or above 0, never decrease and end
+ *   at or below total; it is read on the device only, and one that breaks this is found
+ *   there: nothing is read or written and fa_last_device_error reports FA_ERR_INVALID_ARG.
+ *   Rows outside every sequence are not written.  B <= 1024.
  *
  * in_dtype FA_BF16: q, k, v, o are bf16.  FA_F32: q, k, v are fp32, rounded to bf16 (nearest
- *   even) into the workspace first, and o is written as fp32; fixed length only.  FA_TF32: q, k,
+ *   even) into the workspace first, and o is written as fp32 (fixed or variable length).
+ *   FA_TF32: q, k,
  *   v are fp32, rounded to tf32 (10 mantissa bits, nearest even) into the workspace, and the
  *   products run on the tf32 tensor-core path with P kept in fp32; o fp32; fixed length,
  *   d = 64 (the workspace also holds v transposed).
@@ -201,7 +204,10 @@ FA_EXPORT size_t fa_decode_workspace_size(int B, int Hq, int Lmax, int d, int sp
  * different streams, or on one stream from different threads without ordering) race and
  * give wrong results; order them on one stream.
  * The first call on each device looks up the array's device address (with that device
- * current) and caches it; make that first call before any stream capture.
+ * current) and caches it; make that first call before any stream capture.  The cached
+ * address belongs to that device's context: a process that resets the device
+ * (cudaDeviceReset) or otherwise tears its primary context down must not call this entry
+ * point on that device again, since the library's device memory may then sit elsewhere.
  * Other arguments, results and errors are those of fa_decode. */
 FA_EXPORT fa_status fa_decode_noalloc(const void* q, const void* kcache, const void* vcache, const int32_t* seqlens,
                                       void* o, float* lse, int B, int Hq, int Hkv, int Lmax, int d, float scale,
@@ -241,12 +247,15 @@ FA_EXPORT fa_status fa_decode_paged(const void* q, const void* k_pages, const vo
 FA_EXPORT size_t fa_decode_paged_workspace_size(int B, int Hq, int Hkv, int max_pages_per_seq, int page_size, int d,
                                                 int split_len);
 
-/* Waits for `stream`, then returns FA_ERR_TIMEOUT if any kernel of this library recorded a
+/* Takes the device-side error record (read and cleared in one atomic exchange, on `stream`),
+ * waits for `stream`, and returns FA_ERR_TIMEOUT if any kernel of this library recorded a
  * device-side timeout since the previous call, else FA_ERR_CUDA if a kernel found its shared
  * memory carve-out too small, else FA_ERR_INVALID_ARG if a kernel recorded an invalid
- * device-side input (a block-table entry out of range, a
- * cu_seqlens that fa_bwd_varlen cannot use), and clears the record; FA_ERR_CUDA
- * if the stream reports an error; else FA_OK. */
+ * device-side input (a block-table entry out of range, a cu_seqlens that fa_fwd or
+ * fa_bwd_varlen cannot use); FA_ERR_CUDA if the stream reports an error; else FA_OK.
+ * The record is shared by all kernels of the library on the device (all streams); a timeout
+ * stops only the kernel whose wait ran out, and later launches run normally whether or not
+ * the record has been taken. */
 FA_EXPORT fa_status fa_last_device_error(void* stream);
 
 /* Test support for the failure detection: launches one kernel whose single wait can never be

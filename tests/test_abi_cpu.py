@@ -47,6 +47,9 @@ def test_workspace_sizes(lib):
     assert fa.fa_fwd_workspace_size(2, 12, 12, 2048, 2048, 64, fa.FA_BF16, False) == 0
     n = fa.fa_fwd_workspace_size(1, 1, 1, 128, 128, 64, fa.FA_F32, False)
     assert n >= 3 * 128 * 64 * 2
+    # varlen fp32: Nq = Nk = the packed row count (not multiplied by B)
+    nv = fa.fa_fwd_workspace_size(4, 2, 1, 300, 300, 64, fa.FA_F32, True)
+    assert 300 * 2 * 64 * 2 + 2 * 300 * 64 * 2 <= nv < 4 * 300 * 2 * 64 * 2
     ws = fa.fa_decode_workspace_size(8, 64, 32768, 128, 1024)
     assert ws >= 8 * 64 * 32 * (128 + 2) * 4
     assert fa.fa_decode_workspace_size(0, 64, 32768, 128, 1024) == 0
@@ -70,7 +73,8 @@ def test_fwd_rejects_before_launch(lib):
     assert _fwd_status(lib, scale=float("nan")) == fa.FA_ERR_INVALID_ARG
     assert _fwd_status(lib, B=-1) == fa.FA_ERR_INVALID_ARG
     assert _fwd_status(lib, cu=512, Nq=8, Nk=9) == fa.FA_ERR_INVALID_ARG   # varlen needs Nq == Nk
-    assert _fwd_status(lib, cu=512, dt=1) == fa.FA_ERR_UNSUPPORTED         # fp32 varlen
+    assert _fwd_status(lib, cu=512, dt=1) == fa.FA_ERR_WORKSPACE           # fp32 varlen needs its bf16 copies
+    assert _fwd_status(lib, cu=512, dt=2) == fa.FA_ERR_UNSUPPORTED         # tf32 is fixed length only
     assert _fwd_status(lib, cu=514) == fa.FA_ERR_INVALID_ARG               # misaligned offsets
     assert _fwd_status(lib, dt=1) == fa.FA_ERR_WORKSPACE                   # fp32 needs workspace
     assert _fwd_status(lib, dt=7) == fa.FA_ERR_INVALID_ARG

@@ -55,12 +55,14 @@ def test_decode_small(orc, case):
         assert np.all(host64(o)[empty] == 0) and np.all(np.isneginf(host64(lse)[empty]))
 
 
-def test_decode_split_kv_full(orc):
+@pytest.mark.parametrize("seed_off", [0, 10000, 20000])
+def test_decode_split_kv_full(orc, seed_off):
     """B=8, Hq=64, Hkv=8, d=128, cache 32768, splits of 1024 (the benchmark workload, same
-    launch): every (sequence, head) against the oracle, plus bitwise repeatability."""
+    launch), three seeds: every (sequence, head) against the oracle, plus bitwise
+    repeatability."""
     w = si.WORKLOADS["decode_split_kv"]
     B, Hq, Hkv, L, d, split = w["B"], w["Hq"], w["Hkv"], w["L"], w["d"], w["split"]
-    q, kc, vc = _cache(w["seed"], B, Hq, Hkv, L, d)
+    q, kc, vc = _cache(w["seed"] + seed_off, B, Hq, Hkv, L, d)
     scale = 1.0 / math.sqrt(d)
     qd, kd, vd = dev_bf16(q), dev_bf16(kc), dev_bf16(vc)
     o1, l1 = fa.decode(qd, kd, vd, None, scale=scale, split_len=split)

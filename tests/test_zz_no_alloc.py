@@ -33,18 +33,31 @@ def _noalloc(q, kc, vc, lens, split):
 
 
 def test_noalloc_decode_matches_regular_decode_twice():
+    """Two problems in a row through the shared scratch.  The static-scratch entry point runs
+    the same kernels as fa_decode, so the results must be bitwise equal; the first problem is
+    also checked against the oracle, and the second holds an empty sequence (length 0), whose
+    row must come out as o = 0 and lse = -inf even though the scratch holds the first
+    problem's partials."""
+    import oracle as oracle_mod
+    orc = oracle_mod.get()
     problems = [
         (2101, 4, 32, 4, 5000, 128, [5000, 1, 2600, 4097], 512),
-        (2102, 3, 16, 2, 3000, 64, [1500, 3000, 64], 256),
+        (2102, 3, 16, 2, 3000, 64, [1500, 0, 3000], 256),
     ]
-    for seed, B, Hq, Hkv, L, d, lens, split in problems:
+    for n, (seed, B, Hq, Hkv, L, d, lens, split) in enumerate(problems):
         q, kc, vc, ld = _problem(seed, B, Hq, Hkv, L, d, lens)
         o, lse = _noalloc(q, kc, vc, ld, split)
         o_ref, lse_ref = fa.decode(q, kc, vc, ld, scale=1.0 / math.sqrt(d), split_len=split)
         torch.cuda.synchronize()
         assert fa.fa_last_device_error() == fa.FA_OK
-        check_out(host64(o), host64(o_ref), what="noalloc O")
-        check_lse(host64(lse), host64(lse_ref), what="noalloc lse")
+        assert torch.equal(o, o_ref) and torch.equal(lse, lse_ref), f"problem {n}: differs from fa_decode"
+        if n == 0:
+            o64, l64 = orc.decode(host64(q), host64(kc), host64(vc), np.array(lens, np.int32), 1.0 / math.sqrt(d))
+            check_out(host64(o), o64, what="noalloc O vs oracle")
+            check_lse(host64(lse), l64, what="noalloc lse vs oracle")
+        for b, n_b in enumerate(lens):
+            if n_b == 0:
+                assert np.all(host64(o)[b] == 0) and np.all(np.isneginf(host64(lse)[b]))
 
 
 def test_noalloc_decode_rejects_problems_beyond_its_scratch():
