@@ -741,6 +741,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       constexpr uint32_t idQ = idesc_bf16_f32_mn(D, kBwdQ, true, true);
       const uint32_t kb = smem_u32(sK), vb = smem_u32(sV), qb = smem_u32(sQ), dob = smem_u32(sDO);
       const uint32_t dsb = smem_u32(sDS);
+      const uint64_t dK0 = smem_desc_sw128(kb, 16, 1024), dV0 = smem_desc_sw128(vb, 16, 1024);
+      const uint64_t dKmn = smem_desc_sw128(kb, C::kKPanel, 1024);  // K read d-major (A of dQ^T)
       bool ok = warp_wait(kv_full, 0);
       tc_fence_after();
       for (int t = 0; t <= T && ok; ++t) {
@@ -751,22 +753,27 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
           tc_fence_after();
           const uint32_t qs = qb + slot * C::kQTile, ds = dob + slot * C::kQTile;
           const uint32_t cS = 128 * bb, cDP = 128 * bb + 64;
+          // descriptors built once per pair; a k-step only moves the start address (16-byte
+          // units, no carry: shared addresses are below 2^18 bytes); one elected lane issues
+          // each group of products and its commit
+          const uint64_t dQs = smem_desc_sw128(qs, 16, 1024), dDOs = smem_desc_sw128(ds, 16, 1024);
+          if (elect_one_lane()) {
 #pragma unroll
-          for (int kk = 0; kk < D / 16; ++kk) {
-            const uint32_t ka = (kk >> 2) * C::kKPanel + (kk & 3) * 32;
-            const uint32_t kq = (kk >> 2) * C::kQPanel + (kk & 3) * 32;
-            umma_ss_elect(tmem + cS, smem_desc_sw128(kb + ka, 16, 1024), smem_desc_sw128(qs + kq, 16, 1024), idS,
-                          kk > 0 ? 1u : 0u);
-          }
-          umma_commit_elect(sdp_full + bb);  // the exponentials start while dP^T is formed
+            for (int kk = 0; kk < D / 16; ++kk) {
+              const uint32_t ka = ((kk >> 2) * C::kKPanel + (kk & 3) * 32) >> 4;
+              const uint32_t kq = ((kk >> 2) * C::kQPanel + (kk & 3) * 32) >> 4;
+              mma_ss<0>(tmem + cS, dK0 + ka, dQs + kq, idS, kk > 0 ? 1u : 0u);
+            }
+            umma_commit(sdp_full + bb);  // the exponentials start while dP^T is formed
 #pragma unroll
-          for (int kk = 0; kk < D / 16; ++kk) {
-            const uint32_t ka = (kk >> 2) * C::kKPanel + (kk & 3) * 32;
-            const uint32_t kq = (kk >> 2) * C::kQPanel + (kk & 3) * 32;
-            umma_ss_elect(tmem + cDP, smem_desc_sw128(vb + ka, 16, 1024), smem_desc_sw128(ds + kq, 16, 1024), idS,
-                          kk > 0 ? 1u : 0u);
+            for (int kk = 0; kk < D / 16; ++kk) {
+              const uint32_t ka = ((kk >> 2) * C::kKPanel + (kk & 3) * 32) >> 4;
+              const uint32_t kq = ((kk >> 2) * C::kQPanel + (kk & 3) * 32) >> 4;
+              mma_ss<0>(tmem + cDP, dV0 + ka, dDOs + kq, idS, kk > 0 ? 1u : 0u);
+            }
+            umma_commit(dp_full + bb);
           }
-          umma_commit_elect(dp_full + bb);
+          __syncwarp();
         }
         if (t >= 1) {
           const int tp = t - 1, slot = tp % kBwdSlots, bb = tp & 1;
@@ -774,24 +781,28 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
           tc_fence_after();
           const uint32_t qs = qb + slot * C::kQTile, ds = dob + slot * C::kQTile;
           const uint32_t cS = 128 * bb, cDP = 128 * bb + 64;
+          const uint64_t dDOmn = smem_desc_sw128(ds, C::kQPanel, 1024), dQmn = smem_desc_sw128(qs, C::kQPanel, 1024);
+          const uint64_t dDS = smem_desc_sw128(dsb + bb * C::kDSTile, C::kDSTile, 1024);
+          if (elect_one_lane()) {
 #pragma unroll
-          for (int kk = 0; kk < kBwdQ / 16; ++kk) {
-            const uint32_t acc = (tp > 0 || kk > 0) ? 1u : 0u;
-            // queries 16 kk .. 16 kk + 15: warpgroup kk / 2, P^T at 32 (kk / 2) + 8 (kk % 2), dS^T 16 further
-            const uint32_t pc = cS + 32 * (kk >> 1) + 8 * (kk & 1);
-            umma_ts_elect(tmem + C::kColDV, tmem + pc, smem_desc_sw128(ds + kk * 16 * 128, C::kQPanel, 1024), idAcc,
-                          acc);
-            umma_ts_elect(tmem + C::kColDK, tmem + pc + 16, smem_desc_sw128(qs + kk * 16 * 128, C::kQPanel, 1024),
-                          idAcc, acc);
+            for (int kk = 0; kk < kBwdQ / 16; ++kk) {
+              const uint32_t acc = (tp > 0 || kk > 0) ? 1u : 0u;
+              // queries 16 kk .. 16 kk + 15: warpgroup kk / 2, P^T at 32 (kk / 2) + 8 (kk % 2), dS^T 16 further
+              const uint32_t pc = cS + 32 * (kk >> 1) + 8 * (kk & 1);
+              const uint32_t off = (kk * 16 * 128) >> 4;
+              mma_ts<0>(tmem + C::kColDV, tmem + pc, dDOmn + off, idAcc, acc);
+              mma_ts<0>(tmem + C::kColDK, tmem + pc + 16, dQmn + off, idAcc, acc);
+            }
+            // dQ^T = K^T dS: A = K (keys x d) read d-major, B = dS (keys x queries) query-major
+#pragma unroll
+            for (int kk = 0; kk < kBwdTile / 16; ++kk) {
+              const uint32_t off = (kk * 16 * 128) >> 4;
+              mma_ss<0>(tmem + cDP, dKmn + off, dDS + off, idQ, kk > 0 ? 1u : 0u);
+            }
+            umma_commit(dq_full + bb);
+            umma_commit(q_empty + slot);
           }
-          // dQ^T = K^T dS: A = K (keys x d) read d-major, B = dS (keys x queries) query-major
-#pragma unroll
-          for (int kk = 0; kk < kBwdTile / 16; ++kk)
-            umma_ss_elect(tmem + cDP, smem_desc_sw128(kb + kk * 16 * 128, C::kKPanel, 1024),
-                          smem_desc_sw128(dsb + bb * C::kDSTile + kk * 16 * 128, C::kDSTile, 1024), idQ,
-                          kk > 0 ? 1u : 0u);
-          umma_commit_elect(dq_full + bb);
-          umma_commit_elect(q_empty + slot);
+          __syncwarp();
         }
       }
       umma_commit_elect(acc_done);

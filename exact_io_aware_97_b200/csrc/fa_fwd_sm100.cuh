@@ -68,6 +68,10 @@ constexpr float kRescaleThreshold = 8.0f;
 // SM sub-partition with two softmax warps; measured slower.)
 constexpr int kPChunks = 2;
 constexpr int kChunkKeys = kBN / kPChunks;
+// FP8 only: column pairs (bit e of each group of 8 pairs) whose 2^x runs on the FMA pipe (a
+// polynomial) instead of the special-function unit, in tiles without masked keys.  With its
+// products halved, the fp8 forward is bound by the ex2 rate of the two tiles' softmax steps.
+constexpr uint32_t kFp8FmaExpPairs = 0x11;
 
 
 // Operand kinds of the forward: bf16 (kind::f16); FP8: q, k, v in e4m3 (d = 128 only), the
@@ -473,12 +477,12 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         for (int j = 0; j < nmax && ok; ++j) {
           const uint32_t gv = g + 2 * j + 1;
           const uint32_t gk = g + 2 * j + 2;
+          // both K/V tiles of the step are waited for here, so no data wait sits between the
+          // products of a tile (the producer runs ahead; these waits rarely block)
           if (!wait_full(gv)) { ok = false; break; }
+          if (j + 1 < nmax && !wait_full(gk)) { ok = false; break; }
           if (j < un.n[0] && !pv_step(0, j, gv % NS)) { ok = false; break; }
-          if (j + 1 < nmax) {
-            if (!wait_full(gk)) { ok = false; break; }
-            if (j + 1 < un.n[0]) issue_S(0, gk % NS);
-          }
+          if (j + 1 < nmax && j + 1 < un.n[0]) issue_S(0, gk % NS);
           if (j < un.n[1] && !pv_step(1, j, gv % NS)) { ok = false; break; }
           umma_commit_elect(empty + (gv % NS));
           if (j + 1 < nmax) {
@@ -524,13 +528,19 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       // of nms2) into pk, with the row sum of the unrounded values added to lsum.
       constexpr int kW = FP8 ? kChunkKeys / 4 : (TF32 ? kChunkKeys : kChunkKeys / 2);  // TMEM words
       const uint64_t tau2 = f2(tau, tau);
-      auto make_chunk = [&](const float (&sc)[128], int c, uint64_t nms2, uint32_t (&pk)[kW], uint64_t (&lsum)[2]) {
+      auto make_chunk = [&](const float (&sc)[128], int c, uint64_t nms2, uint32_t (&pk)[kW], uint64_t (&lsum)[2],
+                            bool unmasked) {
 #pragma unroll
         for (int e = 0; e < kChunkKeys / 2; ++e) {
           const int g = c * (kChunkKeys / 2) + e;  // column pair
-          float x0, x1;
+          float x0, x1, p0, p1;
           f2_split(f2_fma(f2(sc[2 * g], sc[2 * g + 1]), tau2, nms2), x0, x1);
-          const float p0 = ex2_approx(x0), p1 = ex2_approx(x1);
+          if (FP8 && ((kFp8FmaExpPairs >> (g & 7)) & 1u) && unmasked) {
+            exp2_poly_x2(x0, x1, p0, p1);
+          } else {
+            p0 = ex2_approx(x0);
+            p1 = ex2_approx(x1);
+          }
           lsum[e & 1] = f2_add(lsum[e & 1], f2(p0, p1));
           if (TF32) {
             pk[2 * e] = __float_as_uint(p0);
@@ -590,12 +600,12 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
           m_tile = row_max128(s) * tau;
           const uint64_t nms2 = f2(-m_ref, -m_ref);
           uint32_t pk[kW];
-          make_chunk(s, 0, nms2, pk, lsum);
+          make_chunk(s, 0, nms2, pk, lsum, true);
           if (!__any_sync(0xffffffffu, m_tile - m_ref > kRescaleThreshold)) {
             publish(0, pk);
 #pragma unroll
             for (int c = 1; c < kPChunks; ++c) {
-              make_chunk(s, c, nms2, pk, lsum);
+              make_chunk(s, c, nms2, pk, lsum, true);
               publish(c, pk);
             }
             float la, lb, lc, ld;
@@ -643,7 +653,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
 #pragma unroll
         for (int c = 0; c < kPChunks; ++c) {
           uint32_t pk[kW];
-          make_chunk(s, c, nms2, pk, lsum);
+          make_chunk(s, c, nms2, pk, lsum, !need_mask);
           publish(c, pk);
         }
         float la, lb, lc, ld;
