@@ -305,7 +305,7 @@ def run_device(args):
     p_o = torch.empty((pB, pHq, pd), dtype=torch.bfloat16, device=dev)
     p_lse = torch.empty((pB, pHq), dtype=torch.float32, device=dev)
     p_ws_bytes = fa.fa_decode_paged_workspace_size(pB, pHq, pHkv, table_np.shape[1], pps, pd, psplit)
-    p_ws = torch.zeros(p_ws_bytes, dtype=torch.uint8, device=dev)  # arrival counters start at zero
+    p_ws = torch.empty(p_ws_bytes, dtype=torch.uint8, device=dev)
 
     if do_fp8:
         f8 = [si.to_e4m3(inputs("fwd", seed, tid, shp)) for tid, shp in
@@ -558,7 +558,7 @@ def run_device(args):
                                       "unit": "GB/s", "frac": round(paged_gbs / peaks["hbm"], 4),
                                       "peak_kind": f"measured copy ({peaks['source']})",
                                       "traffic": ncu_traffic("fa_decode_paged/decode_paged_ragged"),
-                                      "kernels": "fa_decode_split_kernel<128,paged> (merge in-kernel)",
+                                      "kernels": "fa_decode_split_kernel<128,paged> + fa_decode_combine_kernel<128>",
                                       "algorithmic_bytes_per_launch": pkv}},
         "forward_fp8": {"value": round(aggregate_rate(F, world, fp8_mean) / 1e12, 2), "unit": "TFLOP/s",
                         "ms": round(fp8_mean, 4),
@@ -590,7 +590,7 @@ def run_device(args):
         "e2e": {"value": round(world * F / (fwd_e2e_ms * 1e-3) / 1e12, 2), "unit": "TFLOP/s",
                 "h2d_bytes_per_step": h2d_fwd, "d2h_bytes_per_step": d2h_fwd},
         "cpu_baseline": cpu,
-        "gpu_launches": args.steps * (int(do_fwd) * 1 + int(do_dec) * 2 + int(do_paged) * 1 + int(do_bwd) * 3 + int(do_fp8) * 2 + int(do_tf32) * 4
+        "gpu_launches": args.steps * (int(do_fwd) * 1 + int(do_dec) * 2 + int(do_paged) * 2 + int(do_bwd) * 3 + int(do_fp8) * 2 + int(do_tf32) * 4
                                      + int(do_bwdv) * 4 + int(do_mha2k) + int(do_varlen))
         + (0 if args.no_e2e else e2e_steps * (int(do_fwd) * 1 + int(do_dec) * 2)),
         "clocks": clocks.summary(),

@@ -344,8 +344,7 @@ def decode_paged(q, k_pages, v_pages, block_table, seqlens, scale=None, split_le
                  workspace=None, stream=None):
     """O [B,Hq,d], lse [B,Hq] for one query token per sequence over a page pool
     [num_pages, page_size, Hkv, d] addressed by block_table [B, max_pages] (int32) and
-    seqlens [B] (int32).  A workspace passed in must have been zero-filled once (its arrival
-    counters); calls leave it ready for the next call."""
+    seqlens [B] (int32)."""
     import torch
     _require("q", q.dim() == 3, f"[B, Hq, d], got shape {tuple(q.shape)}")
     B, Hq, d = q.shape
@@ -369,7 +368,7 @@ def decode_paged(q, k_pages, v_pages, block_table, seqlens, scale=None, split_le
         lse = torch.empty((B, Hq), dtype=torch.float32, device=q.device)
     ws_bytes = fa_decode_paged_workspace_size(B, Hq, Hkv, maxp, page_size, d, split_len)
     if workspace is None:
-        workspace = torch.zeros(max(ws_bytes, 1), dtype=torch.uint8, device=q.device)
+        workspace = torch.empty(max(ws_bytes, 1), dtype=torch.uint8, device=q.device)
     fa_decode_paged(q, k_pages, v_pages, block_table, seqlens, out, lse, B, Hq, Hkv, num_pages, page_size, maxp, d,
                     scale, split_len, workspace, ws_bytes, stream)
     return out, lse

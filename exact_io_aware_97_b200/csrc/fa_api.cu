@@ -218,6 +218,9 @@ fa_status launch_decode_paged(const void* kp, const void* vp, const DecParams& p
   if (set_smem(ks, smem) != cudaSuccess) return FA_ERR_CUDA;
   dim3 grid(prm.nsplit, prm.Hkv, prm.B);
   ks<<<grid, kDecThreads, smem, st>>>(mk, mv, prm);
+  if (cudaGetLastError() != cudaSuccess) return FA_ERR_CUDA;
+  const int nbh = prm.B * prm.Hq;
+  fa_decode_combine_kernel<D><<<(nbh + 3) / 4, 128, 0, st>>>(prm);
   return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
 
@@ -613,7 +616,7 @@ size_t fa_decode_paged_workspace_size(int B, int Hq, int Hkv, int max_pages_per_
     return 0;
   const int64_t lmax = (int64_t)max_pages_per_seq * page_size;
   if (lmax >= (int64_t(1) << 31)) return 0;
-  return align_up((size_t)B * Hkv * 4, 256) + fa_decode_workspace_size(B, Hq, (int)lmax, d, split_len);
+  return fa_decode_workspace_size(B, Hq, (int)lmax, d, split_len);  // the split partials
 }
 
 fa_status fa_decode_paged(const void* q, const void* k_pages, const void* v_pages, const int32_t* block_table,
@@ -648,8 +651,6 @@ fa_status fa_decode_paged(const void* q, const void* k_pages, const void* v_page
   prm.seqlens = seqlens;
   prm.o = static_cast<__nv_bfloat16*>(o);
   prm.lse = lse;
-  prm.counters = reinterpret_cast<uint32_t*>(ws);
-  ws += align_up((size_t)B * Hkv * 4, 256);
   prm.ws_acc = reinterpret_cast<float*>(ws);
   prm.ws_ml = reinterpret_cast<float*>(ws + align_up(parts * d * 4, 256));
   prm.block_table = block_table;

@@ -8,15 +8,15 @@
 // accumulator acc_s = sum_j 2^(t_j - m_s) v_j.  A second kernel merges the splits with the
 // rule of "FlashAttention notes" section 4 (m = max m_s, l = sum 2^(m_s - m) l_s, and the
 // accumulators with the same weights) ("FlashAttention-3 (FA-3)", section 4, FlashDecoding).
+// (Merging in the split kernel instead, by the last CTA of each (sequence, KV head) to finish,
+// measured slower: those merges run serially at the end of the grid, while the combine kernel
+// spreads them over all SMs.)
 //
 // Paged caches ("LLM basics: from Attention to FlashAttention", chapter 2 section 8,
 // PagedAttention): the cache is a pool of fixed-size pages, and a per-sequence block table
 // maps logical page t / page_size of a sequence to a physical page, so token t sits at row
 // t % page_size of that page.  The paged kernel fetches each 64-row stage as whole pages
-// (or one 64-row part of a larger page) through the table, and merges the splits itself:
-// every split CTA publishes its partial, counts itself in on a per-(sequence, KV head)
-// counter, and the CTA that arrives last merges all partials of that group (no CTA waits
-// for another, and no second launch).  A sequence that fits one split skips the partial.
+// (or one 64-row part of a larger page) through the table.
 //
 // The split kernel is bound by HBM bandwidth: K and V are read once.  Tiles of 64 cache rows
 // arrive by TMA (128-byte swizzle, evict-first) in a 3- or 4-stage ring fed by a producer
@@ -38,7 +38,6 @@ struct DecParams {
   float* ws_ml;   // [B, Hq, nsplit, 2]  (m in base-2 units, l)
   // paged caches only
   const int32_t* block_table;  // [B, max_pages]
-  uint32_t* counters;          // [B, Hkv] split arrivals; zero between calls
   int max_pages, page_shift, page_box, num_pages;
   int B, Hq, Hkv, G, Lmax, split_len, nsplit;
   float tau;
@@ -91,21 +90,9 @@ __device__ __forceinline__ int dec_seqlen(const DecParams& p, int b) {
   return max(0, min(L, p.Lmax));
 }
 
-// Writes o (bf16) and lse of query head h of sequence b from the merged numerator a / l and
-// the base-2 max m.  An empty row (l = 0) gives o = 0 and lse = -inf.
-__device__ __forceinline__ void dec_store_row4(const DecParams& p, int b, int h, int col, float4 a, float m, float l,
-                                               int D) {
-  const float inv = l > 0.f ? 1.f / l : 0.f;
-  uint2 w;
-  w.x = pack_bf16x2(a.x * inv, a.y * inv);
-  w.y = pack_bf16x2(a.z * inv, a.w * inv);
-  *reinterpret_cast<uint2*>(p.o + ((size_t)b * p.Hq + h) * D + col) = w;
-  if (col == 0 && p.lse != nullptr) p.lse[(size_t)b * p.Hq + h] = l > 0.f ? (m + log2f(l)) * kLn2 : -INFINITY;
-}
-
-// PAGED = false: contiguous caches [B, Lmax, Hkv, D]; partials of every split go to the
-// workspace and fa_decode_combine_kernel merges them.  PAGED = true: page pool
-// [num_pages, page_size, Hkv, D] through the block table, merged in this kernel.
+// PAGED = false: contiguous caches [B, Lmax, Hkv, D].  PAGED = true: page pool
+// [num_pages, page_size, Hkv, D] through the block table.  Either way the partial of every
+// split goes to the workspace and fa_decode_combine_kernel merges them.
 template <int D, bool PAGED>
 __global__ void __launch_bounds__(kDecThreads)
     fa_decode_split_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
@@ -118,14 +105,7 @@ __global__ void __launch_bounds__(kDecThreads)
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int G = p.G;
   const int h0 = kvh * G;
-  if (key_begin >= seqlen) {
-    // Empty split.  Unpaged, the combine kernel never reads it.  Paged, an empty sequence
-    // still needs its output, which the first split writes.
-    if (PAGED && split == 0 && warp < kDecComputeWarps)
-      for (int idx = threadIdx.x; idx < G * (D / 4); idx += kDecComputeWarps * 32)
-        dec_store_row4(p, b, h0 + idx / (D / 4), 4 * (idx % (D / 4)), make_float4(0.f, 0.f, 0.f, 0.f), 0.f, 0.f, D);
-    return;
-  }
+  if (key_begin >= seqlen) return;  // empty split: the combine kernel never reads it
   const int nkeys = min(p.split_len, seqlen - key_begin);
   const int nst = (nkeys + kDecKeys - 1) / kDecKeys;
 
@@ -133,7 +113,6 @@ __global__ void __launch_bounds__(kDecThreads)
   uint8_t* ring = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* full = reinterpret_cast<uint64_t*>(ring + NS * C::kStageBytes);
   uint64_t* empty = full + NS;
-  uint32_t* last_flag = reinterpret_cast<uint32_t*>(empty + NS);
   if (threadIdx.x == 0) {
     for (int s = 0; s < NS; ++s) {
       mbar_init(full + s, 1);
@@ -330,7 +309,6 @@ __global__ void __launch_bounds__(kDecThreads)
   }
   asm volatile("bar.sync 1, %0;" ::"n"(kDecComputeWarps * 32) : "memory");
   const size_t part0 = ((size_t)b * p.Hq + h0) * p.nsplit + split;  // partial of head h0
-  const int ns_b = (seqlen + p.split_len - 1) / p.split_len;       // splits of this sequence
   for (int idx = threadIdx.x; idx < G * (D / 4); idx += kDecComputeWarps * 32) {
     const int row = idx / (D / 4), col = 4 * (idx - row * (D / 4));
     float M = -INFINITY;
@@ -349,74 +327,12 @@ __global__ void __launch_bounds__(kDecThreads)
       A.z += e * x.z;
       A.w += e * x.w;
     }
-    if (PAGED && ns_b == 1) {  // the only split of its sequence: the result is final
-      dec_store_row4(p, b, h0 + row, col, A, M, L, D);
-      continue;
-    }
     const size_t part = part0 + (size_t)row * p.nsplit;
     *reinterpret_cast<float4*>(p.ws_acc + part * D + col) = A;
     if (col == 0) {
       p.ws_ml[part * 2] = M;
       p.ws_ml[part * 2 + 1] = L;
     }
-  }
-  if (!PAGED || ns_b == 1) return;
-
-  // Count this split in; the last of the sequence's splits to arrive merges them all.  Each
-  // writer fences its partial before the CTA barrier, and the counting thread's atomic is
-  // ordered after that barrier, so a CTA that sees the final count sees every partial.
-  __threadfence();
-  asm volatile("bar.sync 1, %0;" ::"n"(kDecComputeWarps * 32) : "memory");
-  uint32_t* counter = p.counters + (size_t)b * p.Hkv + kvh;
-  if (threadIdx.x == 0) {
-    const uint32_t before = atomicAdd(counter, 1u);
-    const bool last = before + 1 == (uint32_t)ns_b;
-    if (last) *counter = 0u;  // every split of this call has counted; ready for the next call
-    __threadfence();
-    *last_flag = last ? 1u : 0u;
-  }
-  asm volatile("bar.sync 1, %0;" ::"n"(kDecComputeWarps * 32) : "memory");
-  if (*last_flag == 0u) return;
-
-  // Merge ("FlashAttention notes", section 4): m = max_s m_s, l = sum_s 2^(m_s - m) l_s,
-  // o = sum_s 2^(m_s - m) acc_s / l.  Partials were written by other SMs: read through L2.
-  float* sm_M = sm_l + kDecComputeWarps * 16;  // [16]
-  float* sm_L = sm_M + 16;                     // [16]
-  const size_t bh0 = ((size_t)b * p.Hq + h0) * p.nsplit;
-  for (int row = warp; row < G; row += kDecComputeWarps) {
-    const float* ml = p.ws_ml + (bh0 + (size_t)row * p.nsplit) * 2;
-    float M = -INFINITY;
-    for (int s = lane; s < ns_b; s += 32) M = fmaxf(M, __ldcg(ml + 2 * s));
-#pragma unroll
-    for (int off = 16; off > 0; off >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
-    float L = 0.f;
-    for (int s = lane; s < ns_b; s += 32) {
-      const float ms = __ldcg(ml + 2 * s);
-      L += (ms == -INFINITY) ? 0.f : ex2_approx(ms - M) * __ldcg(ml + 2 * s + 1);
-    }
-#pragma unroll
-    for (int off = 16; off > 0; off >>= 1) L += __shfl_xor_sync(0xffffffffu, L, off);
-    if (lane == 0) {
-      sm_M[row] = M;
-      sm_L[row] = L;
-    }
-  }
-  asm volatile("bar.sync 1, %0;" ::"n"(kDecComputeWarps * 32) : "memory");
-  for (int idx = threadIdx.x; idx < G * (D / 4); idx += kDecComputeWarps * 32) {
-    const int row = idx / (D / 4), col = 4 * (idx - row * (D / 4));
-    const size_t base = bh0 + (size_t)row * p.nsplit;
-    const float M = sm_M[row];
-    float4 A = make_float4(0.f, 0.f, 0.f, 0.f);
-    for (int s = 0; s < ns_b; ++s) {
-      const float ms = __ldcg(p.ws_ml + (base + s) * 2);
-      const float e = (ms == -INFINITY) ? 0.f : ex2_approx(ms - M);
-      const float4 x = __ldcg(reinterpret_cast<const float4*>(p.ws_acc + (base + s) * D + col));
-      A.x += e * x.x;
-      A.y += e * x.y;
-      A.z += e * x.z;
-      A.w += e * x.w;
-    }
-    dec_store_row4(p, b, h0 + row, col, A, M, sm_L[row], D);
   }
 }
 

@@ -215,8 +215,7 @@ FA_EXPORT fa_status fa_decode_noalloc(const void* q, const void* kcache, const v
 
 /* Split-KV decode over a paged KV cache ("LLM basics: from Attention to FlashAttention",
  * chapter 2 section 8, PagedAttention: fixed-size pages of the cache, mapped from each
- * sequence's logical pages by a block table), with the split merge done inside the same
- * launch by the last split of each (sequence, KV head) to finish.
+ * sequence's logical pages by a block table); the splits are merged as in fa_decode.
  *
  * q [B, Hq, d] bf16; k_pages and v_pages [num_pages, page_size, Hkv, d] bf16 (the page
  * pool); block_table: device int32 [B, max_pages_per_seq], entry (b, t) = the physical page
@@ -232,12 +231,8 @@ FA_EXPORT fa_status fa_decode_noalloc(const void* q, const void* kcache, const v
  * num_pages * page_size < 2^31.
  * A block-table entry outside [0, num_pages) is read as page 0 and recorded on the device;
  * fa_last_device_error then returns FA_ERR_INVALID_ARG.
- * workspace: at least fa_decode_paged_workspace_size(...) bytes.  Its first
- * 4 * B * Hkv bytes (rounded up to 256) are arrival counters that MUST be zero before the
- * first call with this workspace (e.g. allocate it zero-filled); every call that completes
- * leaves them zero again, so the same workspace serves later calls without clearing.  After
- * a call that reported FA_ERR_TIMEOUT, zero it again.  Calls sharing a workspace must not
- * overlap on the GPU. */
+ * workspace: at least fa_decode_paged_workspace_size(...) bytes (the split partials); its
+ * contents need not be initialised.  Calls sharing a workspace must not overlap on the GPU. */
 FA_EXPORT fa_status fa_decode_paged(const void* q, const void* k_pages, const void* v_pages,
                                     const int32_t* block_table, const int32_t* seqlens, void* o, float* lse, int B,
                                     int Hq, int Hkv, int num_pages, int page_size, int max_pages_per_seq, int d,

@@ -128,10 +128,12 @@ def test_decode_paged_rejects_before_launch(lib):
     assert _paged_status(lib, B=0) == fa.FA_OK
 
 
-def test_decode_paged_workspace_holds_counters_and_partials(lib):
+def test_decode_paged_workspace_holds_the_partials(lib):
     B, Hq, Hkv, maxp, ps, d, split = 16, 64, 8, 2048, 16, 128, 1024
     n = fa.fa_decode_paged_workspace_size(B, Hq, Hkv, maxp, ps, d, split)
-    assert n >= B * Hkv * 4 + fa.fa_decode_workspace_size(B, Hq, maxp * ps, d, split)
+    nsplit = (maxp * ps + split - 1) // split
+    assert n >= B * Hq * nsplit * (d + 2) * 4
+    assert n == fa.fa_decode_workspace_size(B, Hq, maxp * ps, d, split)
     assert fa.fa_decode_paged_workspace_size(0, Hq, Hkv, maxp, ps, d, split) == 0
 
 

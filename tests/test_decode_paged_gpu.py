@@ -62,8 +62,9 @@ def test_decode_paged_small(orc, case):
     seed, B, Hq, Hkv, d, ps, lens, split, extra = case
     q, kp, vp, table, lens_np = _problem(seed, B, Hq, Hkv, d, ps, lens, extra)
     scale = 1.0 / math.sqrt(d)
-    ws = torch.zeros(fa.fa_decode_paged_workspace_size(B, Hq, Hkv, table.shape[1], ps, d, split),
-                     dtype=torch.uint8, device="cuda")
+    # a workspace full of garbage bytes: nothing in it needs initialising
+    ws = torch.full((fa.fa_decode_paged_workspace_size(B, Hq, Hkv, table.shape[1], ps, d, split),), 0xFF,
+                    dtype=torch.uint8, device="cuda")
     o, lse = _run(q, kp, vp, table, lens_np, scale, split, ws)
     torch.cuda.synchronize()
     assert fa.fa_last_device_error() == fa.FA_OK
@@ -73,15 +74,14 @@ def test_decode_paged_small(orc, case):
     empty = lens_np == 0
     if empty.any():
         assert np.all(host64(o)[empty] == 0) and np.all(np.isneginf(host64(lse)[empty]))
-    # the arrival counters are back at zero: the same workspace gives the same bits again
+    # the same workspace, reused, gives the same bits again
     o2, lse2 = _run(q, kp, vp, table, lens_np, scale, split, ws)
     torch.cuda.synchronize()
     assert torch.equal(o, o2) and torch.equal(lse, lse2)
-    assert int(ws[: B * Hkv * 4].view(torch.int32).abs().sum()) == 0
 
 
 def test_decode_paged_workspace_reused_across_problems(orc):
-    """One zero-filled workspace serves a sequence of different problems."""
+    """One workspace serves a sequence of different problems."""
     ws = torch.zeros(8 << 20, dtype=torch.uint8, device="cuda")
     for seed, B, Hq, Hkv, d, ps, lens, split, extra in [CASES[0], CASES[3], CASES[1], CASES[0]]:
         q, kp, vp, table, lens_np = _problem(seed, B, Hq, Hkv, d, ps, lens, extra)
