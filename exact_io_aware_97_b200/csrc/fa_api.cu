@@ -152,6 +152,20 @@ bool make_map_f32(CUtensorMap* map, const void* base, const cuuint64_t (&dims)[3
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// Dense bf16 output [rows, heads, D] as the TMA store target of the forward epilogue: box of
+// 16 columns x 1 head x 32 rows (one softmax warp's rows) with the 32-byte swizzle.
+bool make_map_o(CUtensorMap* map, const void* base, int D, int heads, int64_t rows) {
+  EncodeTiledFn enc = get_encode_fn();
+  if (!enc || rows <= 0 || (reinterpret_cast<uintptr_t>(base) & 15u) != 0) return false;
+  cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)heads, (cuuint64_t)rows};
+  cuuint64_t strides[2] = {(cuuint64_t)D * 2, (cuuint64_t)heads * D * 2};
+  cuuint32_t box[3] = {16, 1, 32};
+  cuuint32_t estr[3] = {1, 1, 1};
+  return enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_32B, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 int sm_count_cached() {
   static int counts[64] = {0};
   int dev = 0;
@@ -180,13 +194,18 @@ fa_status launch_fwd(const void* q, const void* k, const void* v, const FwdParam
   if (!make_map(&mq, q, D, prm.Hq, rows_q, kBM, q_stride) || !make_map(&mk, k, D, prm.Hkv, rows_k, kBN, kv_stride) ||
       !make_map(&mv, v, D, prm.Hkv, rows_k, kBN, kv_stride))
     return FA_ERR_CUDA;
+  // bf16 O goes out through TMA stores when it can be described (16-byte aligned base); the
+  // kernel writes per lane otherwise (and always for fp32 O)
+  FwdParams p2 = prm;
+  CUtensorMap mo = mq;
+  p2.o_tma = (!F32 && make_map_o(&mo, prm.o, D, prm.Hq, rows_q)) ? 1 : 0;
   auto kern = fa_fwd_kernel<D, F32>;
   const int smem = FwdCfg<D>::kSmemBytes;
   if (set_smem(kern, smem) != cudaSuccess) return FA_ERR_CUDA;
   const int sms = sm_count_cached();
   if (sms <= 0) return FA_ERR_CUDA;
   const int grid = (units > 0) ? std::min(units, sms) : sms;
-  kern<<<grid, kFwdThreads, smem, st>>>(mq, mk, mv, prm);
+  kern<<<grid, kFwdThreads, smem, st>>>(mq, mk, mv, mo, p2);
   return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
 
@@ -376,7 +395,7 @@ fa_status fwd_tf32(const void* q, const void* k, const void* v, void* o, float* 
   if (set_smem(kern, smem) != cudaSuccess) return FA_ERR_CUDA;
   const int sms = sm_count_cached();
   if (sms <= 0) return FA_ERR_CUDA;
-  kern<<<std::min((int)units64, sms), kFwdThreads, smem, st>>>(mq, mk, mv, prm);
+  kern<<<std::min((int)units64, sms), kFwdThreads, smem, st>>>(mq, mk, mv, mq, prm);  // fp32 O: per-lane stores
   return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
 
@@ -516,13 +535,15 @@ fa_status fa_fwd_fp8(const void* q, const void* k, const void* v, void* o, float
   if (!make_map_u8(&mq, q, dq3, sq2, box_rows) || !make_map_u8(&mk, k, dk3, sk2, box_rows) ||
       !make_map_u8(&mv, Nk > 0 ? (const void*)vt : k, dv3, sv2, box_vt))
     return FA_ERR_CUDA;
+  CUtensorMap mo = mq;
+  prm.o_tma = make_map_o(&mo, o, 128, Hq, rows_q) ? 1 : 0;
   auto kern = fa_fwd_kernel<128, false, kKindFP8>;
   const int smem = FwdCfg<128, kKindFP8>::kSmemBytes;
   if (set_smem(kern, smem) != cudaSuccess) return FA_ERR_CUDA;
   const int sms = sm_count_cached();
   if (sms <= 0) return FA_ERR_CUDA;
   const int units = (int)units64;
-  kern<<<std::min(units, sms), kFwdThreads, smem, st>>>(mq, mk, mv, prm);
+  kern<<<std::min(units, sms), kFwdThreads, smem, st>>>(mq, mk, mv, mo, prm);
   return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
 

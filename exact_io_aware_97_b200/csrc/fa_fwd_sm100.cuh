@@ -46,6 +46,7 @@ struct FwdParams {
   float tau;      // scale * log2(e) (fp8: times the q and k dequantisation factors)
   float o_scale;  // multiplies O at the end (fp8: the v dequantisation factor; else 1)
   int T;          // fixed length: 256-row units per (sequence, head)
+  int o_tma;      // bf16 O written through shared memory by TMA stores (tmO describes o)
 };
 
 constexpr int kBM = 128;        // query rows per tile
@@ -91,10 +92,14 @@ struct FwdCfg {
   static constexpr int kStages = KIND == kKindTF32 ? 4 : ((KIND == kKindFP8 || D == 64) ? 8 : 4);
   static constexpr int kQBytes = 2 * kTileBytes;
   static constexpr int kRingBytes = kStages * kTileBytes;
+  // Epilogue staging: per softmax warp two 1 KB boxes of 32 rows x 16 bf16 columns (32-byte
+  // swizzle), each stored to O by TMA while the warp fills the other.
+  static constexpr int kStageBoxBytes = 32 * 32;
+  static constexpr int kStageBytes = 8 * 2 * kStageBoxBytes;
   static constexpr int kNumBars = 2 + 2 * kStages + 6 + 2 * kPChunks;
   static constexpr int kBarBytes = kNumBars * 8 + 16;
   static constexpr int kSchedBytes = kMaxVarlenB * 2 + kMaxVarlenT * 4 + 16;
-  static constexpr int kSmemBytes = 1024 + kQBytes + kRingBytes + kBarBytes + kSchedBytes;
+  static constexpr int kSmemBytes = 1024 + kQBytes + kRingBytes + kStageBytes + kBarBytes + kSchedBytes;
   static constexpr uint32_t kTmemCols = 512;
   static constexpr uint32_t kColO = 256;
 };
@@ -208,7 +213,8 @@ __device__ __forceinline__ float row_max128(const float (&s)[128]) {
 template <int D, bool OUT_F32, int KIND = kKindBF16>
 __global__ void __launch_bounds__(kFwdThreads, 1)
     fa_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
-                  const __grid_constant__ CUtensorMap tmV, const FwdParams p) {
+                  const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmO,
+                  const FwdParams p) {
   constexpr bool FP8 = KIND == kKindFP8, TF32 = KIND == kKindTF32;
   static_assert(!FP8 || (D == 128 && !OUT_F32), "fp8 forward: d = 128, bf16 output");
   static_assert(!TF32 || (D == 64 && OUT_F32), "tf32 forward: d = 64, fp32 output");
@@ -218,7 +224,8 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sQ = smem;
   uint8_t* sRing = smem + C::kQBytes;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(sRing + C::kRingBytes);
+  uint8_t* sStage = sRing + C::kRingBytes;  // 1024-byte aligned (Q and ring are multiples of 1 KB)
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sStage + C::kStageBytes);
   uint64_t* q_full = bars + 0;
   uint64_t* q_empty = bars + 1;
   uint64_t* full = bars + 2;
@@ -258,6 +265,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
     prefetch_tensormap(&tmK);
     prefetch_tensormap(&tmV);
   }
+  if (!OUT_F32 && p.o_tma && warp == 0 && lane == 0) prefetch_tensormap(&tmO);
   if (warp == 8) {
     tmem_alloc(tmem_slot, C::kTmemCols);
     tmem_relinquish();
@@ -672,7 +680,14 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       const bool row_ok = row < un.nq;
       const float inv_l = l > 0.f ? p.o_scale / l : 0.f;
       const size_t orow = ((size_t)(un.q_start + row) * p.Hq + un.h) * D;
-#pragma unroll
+      // A warp whose 32 rows all lie in the sequence writes O by TMA: its rows go to a 1 KB
+      // box of shared memory 16 columns at a time (two boxes in turn, the 32-byte swizzle
+      // keeps the row-per-lane writes free of bank conflicts) and one lane stores each box.
+      // Per-lane global stores would put 32 rows' partial sectors into every instruction.
+      const bool tma_o = !OUT_F32 && p.o_tma && __all_sync(0xffffffffu, row_ok);
+      // One copy of the chunk code: the epilogue runs once per unit, its instructions cold in
+      // the instruction cache, so a rolled loop fetches them once rather than D / 32 times.
+#pragma unroll 1
       for (int c = 0; c < D / 32; ++c) {
         uint32_t ov[32];
         if (n > 0) {
@@ -688,7 +703,34 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
           __syncwarp();
           if (lane == 0) mbar_arrive(o_free + i);
         }
-        if (row_ok) {
+        if (tma_o) {
+#pragma unroll
+          for (int hb = 0; hb < 2; ++hb) {
+            uint8_t* box = sStage + ((warp & 7) * 2 + hb) * C::kStageBoxBytes;
+            if (lane == 0) bulk_wait_group_read1();  // this box's previous store has read it
+            __syncwarp();
+            uint4 w0, w1;
+            const int e0 = 16 * hb;
+            w0.x = pack_bf16x2(__uint_as_float(ov[e0 + 0]) * inv_l, __uint_as_float(ov[e0 + 1]) * inv_l);
+            w0.y = pack_bf16x2(__uint_as_float(ov[e0 + 2]) * inv_l, __uint_as_float(ov[e0 + 3]) * inv_l);
+            w0.z = pack_bf16x2(__uint_as_float(ov[e0 + 4]) * inv_l, __uint_as_float(ov[e0 + 5]) * inv_l);
+            w0.w = pack_bf16x2(__uint_as_float(ov[e0 + 6]) * inv_l, __uint_as_float(ov[e0 + 7]) * inv_l);
+            w1.x = pack_bf16x2(__uint_as_float(ov[e0 + 8]) * inv_l, __uint_as_float(ov[e0 + 9]) * inv_l);
+            w1.y = pack_bf16x2(__uint_as_float(ov[e0 + 10]) * inv_l, __uint_as_float(ov[e0 + 11]) * inv_l);
+            w1.z = pack_bf16x2(__uint_as_float(ov[e0 + 12]) * inv_l, __uint_as_float(ov[e0 + 13]) * inv_l);
+            w1.w = pack_bf16x2(__uint_as_float(ov[e0 + 14]) * inv_l, __uint_as_float(ov[e0 + 15]) * inv_l);
+            // row = lane, 32 bytes; 16-byte half h sits at h ^ bit 2 of the row (32-byte swizzle)
+            const int sw = (lane >> 2) & 1;
+            *reinterpret_cast<uint4*>(box + lane * 32 + (sw << 4)) = w0;
+            *reinterpret_cast<uint4*>(box + lane * 32 + ((sw ^ 1) << 4)) = w1;
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) {
+              tma_store_3d(&tmO, box, 32 * c + e0, un.h, un.q_start + row);
+              bulk_commit_group();
+            }
+          }
+        } else if (row_ok) {
           if (OUT_F32) {
             float4* dst = reinterpret_cast<float4*>(reinterpret_cast<float*>(p.o) + orow + 32 * c);
 #pragma unroll
@@ -716,6 +758,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         p.lse[li] = v;
       }
     }
+    if (lane == 0) bulk_wait_group0();  // O boxes stored before the CTA's shared memory goes
   }
 
   tc_fence_before();
