@@ -262,9 +262,13 @@ fa_status launch_bwd(const void* q, const void* k, const void* v, const BwdParam
   if (pre_blocks > 0) fa_bwd_pre_kernel<D><<<pre_blocks, 256, 0, st>>>(prm);
   if (cudaGetLastError() != cudaSuccess) return FA_ERR_CUDA;
   if (rows_k > 0 && (varlen || prm.Nk > 0)) {
-    // varlen: one CTA index per tile of any sequence (bounded by ntiles; the kernels find
-    // the sequence and leave indices past the last tile idle)
-    const dim3 grid = varlen ? dim3(prm.ntiles, prm.Hkv, 1) : dim3((prm.Nk + kBwdTile - 1) / kBwdTile, prm.Hkv, prm.B);
+    // one CTA per (key tile, K/V head, sequence), tile-major (the kernels' bwd_cta_coords);
+    // varlen: a tile number over all sequences (bounded by ntiles; the kernels find the
+    // sequence and leave numbers past the last tile idle)
+    const long long ctas = varlen ? (long long)prm.ntiles * prm.Hkv
+                                  : (long long)((prm.Nk + kBwdTile - 1) / kBwdTile) * prm.Hkv * prm.B;
+    if (ctas >= (1ll << 31)) return FA_ERR_UNSUPPORTED;
+    const dim3 grid((unsigned)ctas);
     if (D == 128) {
       // pairs of 64 queries, two in flight: Q and dO maps with 64-row boxes
       CUtensorMap mq64, mdo64;

@@ -134,6 +134,20 @@ __device__ __forceinline__ bool bwd_locate(const BwdParams& p, int x, int z, Bwd
   return true;
 }
 
+// CTA index -> (key tile number x, K/V head, sequence z) of the main kernels' 1-D grid.
+// Tile-major with the heads (and at fixed length the sequences) varying fastest: in a causal
+// backward the first key tiles of a sequence see the most query tiles, so the longest CTAs
+// are launched first (close to a longest-first list schedule); head-major order would start
+// the last head's long tiles only after every other head's work (8K causal: ~20 % longer).
+__device__ __forceinline__ void bwd_cta_coords(const BwdParams& p, int& x, int& kvh, int& z) {
+  const int per = p.Hkv * (p.cu == nullptr ? p.B : 1);
+  const int L = (int)blockIdx.x;
+  x = L / per;
+  const int r = L - x * per;
+  kvh = r % p.Hkv;
+  z = r / p.Hkv;
+}
+
 // ------------------------------------------------------------------ varlen: tile prefix sums
 // One block: tiles[b] = sum over sequences before b of ceil(len / 128).  cu must start at or
 // above 0, never decrease and end at or below total; otherwise every entry is 0 (no CTA of
@@ -303,8 +317,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   BwdSeq sq;
-  if (!bwd_locate(p, blockIdx.x, blockIdx.z, sq)) return;  // varlen: no tile of this index
-  const int kvh = blockIdx.y;
+  int cta_x, kvh, cta_z;
+  bwd_cta_coords(p, cta_x, kvh, cta_z);
+  if (!bwd_locate(p, cta_x, cta_z, sq)) return;  // varlen: no tile of this index
   const int Nq = sq.nq, Nk = sq.nk;
   const int n0 = sq.tile * kBwdTile;
   const int diag = Nk - Nq;  // causal: key j is allowed for query i iff j <= i + diag
@@ -649,8 +664,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   BwdSeq sq;
-  if (!bwd_locate(p, blockIdx.x, blockIdx.z, sq)) return;  // varlen: no tile of this index
-  const int kvh = blockIdx.y;
+  int cta_x, kvh, cta_z;
+  bwd_cta_coords(p, cta_x, kvh, cta_z);
+  if (!bwd_locate(p, cta_x, cta_z, sq)) return;  // varlen: no tile of this index
   const int Nq = sq.nq, Nk = sq.nk;
   const int n0 = sq.tile * kBwdTile;
   const int diag = Nk - Nq;
