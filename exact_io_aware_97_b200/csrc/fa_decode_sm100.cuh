@@ -129,7 +129,31 @@ __global__ void __launch_bounds__(kDecThreads)
       prefetch_tensormap(&tmV);
       const uint64_t pol = policy_evict_first();
       const int row_base = b * p.Lmax + key_begin;
+      // paged: page_box = min(page_size, 64) rows per copy, so a stage takes at most four
+      // copies and no copy straddles a page.  Copies past the sequence end re-read its last
+      // page (those rows are masked and their V rows zeroed before use).  The block-table
+      // entries of stage s + 1 are loaded while stage s is waited for and issued, so the
+      // table's latency stays off the copy stream.
+      const int box = PAGED ? p.page_box : kDecKeys;
+      const int ps = PAGED ? (1 << p.page_shift) : 1;
+      auto stage_tok = [&](int s, int t) {
+        const int tok = key_begin + s * kDecKeys + t;
+        return tok < seqlen ? tok : ((seqlen - 1) & ~(box - 1));
+      };
+      const int* bt = PAGED ? p.block_table + (size_t)b * p.max_pages : nullptr;
+      int pages[4] = {0, 0, 0, 0};
+      if (PAGED) {
+#pragma unroll
+        for (int k = 0; k < 4; ++k)
+          if (k * box < kDecKeys) pages[k] = __ldg(bt + (stage_tok(0, k * box) >> p.page_shift));
+      }
       for (int s = 0; s < nst; ++s) {
+        const int cur[4] = {pages[0], pages[1], pages[2], pages[3]};
+        if (PAGED && s + 1 < nst) {
+#pragma unroll
+          for (int k = 0; k < 4; ++k)
+            if (k * box < kDecKeys) pages[k] = __ldg(bt + (stage_tok(s + 1, k * box) >> p.page_shift));
+        }
         const int slot = s % NS;
         if (s >= NS && !mbar_wait(empty + slot, ((s / NS) - 1) & 1)) break;
         mbar_arrive_expect_tx(full + slot, C::kStageBytes);
@@ -141,15 +165,12 @@ __global__ void __launch_bounds__(kDecThreads)
                              full + slot, pol);
           }
         } else {
-          // page_box = min(page_size, 64) rows per copy; a stage never straddles a page
-          // boundary inside one copy.  Copies past the sequence end re-read its last page
-          // (those rows are masked and their V rows zeroed before use).
-          const int box = p.page_box;
-          const int ps = 1 << p.page_shift;
-          for (int t = 0; t < kDecKeys; t += box) {
-            int tok = key_begin + s * kDecKeys + t;
-            if (tok >= seqlen) tok = (seqlen - 1) & ~(box - 1);
-            int page = __ldg(p.block_table + (size_t)b * p.max_pages + (tok >> p.page_shift));
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            const int t = k * box;
+            if (t >= kDecKeys) break;
+            const int tok = stage_tok(s, t);
+            int page = cur[k];
             if (page < 0 || page >= p.num_pages) {
               atomicOr(&g_error_word, kErrBadPage);
               page = 0;
