@@ -135,17 +135,26 @@ __device__ __forceinline__ bool bwd_locate(const BwdParams& p, int x, int z, Bwd
 }
 
 // CTA index -> (key tile number x, K/V head, sequence z) of the main kernels' 1-D grid.
-// Tile-major with the heads (and at fixed length the sequences) varying fastest: in a causal
-// backward the first key tiles of a sequence see the most query tiles, so the longest CTAs
-// are launched first (close to a longest-first list schedule); head-major order would start
-// the last head's long tiles only after every other head's work (8K causal: ~20 % longer).
+// K/V heads go in groups of kBwdHeadGroup; within a group the order is tile-major with the
+// group's heads (and at fixed length the sequences) varying fastest.  In a causal backward
+// the first key tiles of a sequence see the most query tiles, so each group launches its
+// longest CTAs first (close to a longest-first list schedule), while the CTAs in flight
+// share few heads, so that their Q, dO and fp32 dQ-accumulator rows mostly stay in L2.
+// Measured on the 8K GQA causal backward (Hkv = 8), groups of 1 (head-major) / 2 / 4 / 8:
+// 3.72 / 3.21 / 3.16 / 3.22 ms with 1.19 / 1.77 / 3.74 / 6.48 GB of DRAM traffic.
+constexpr int kBwdHeadGroup = 2;
 __device__ __forceinline__ void bwd_cta_coords(const BwdParams& p, int& x, int& kvh, int& z) {
-  const int per = p.Hkv * (p.cu == nullptr ? p.B : 1);
+  const int Z = p.cu == nullptr ? p.B : 1;
+  const int X = p.cu == nullptr ? (p.Nk + kBwdTile - 1) / kBwdTile : p.ntiles;
+  const int hg = min(kBwdHeadGroup, p.Hkv);
   const int L = (int)blockIdx.x;
-  x = L / per;
-  const int r = L - x * per;
-  kvh = r % p.Hkv;
-  z = r / p.Hkv;
+  const int gi = L / (X * hg * Z);
+  const int r = L - gi * (X * hg * Z);
+  const int sz = min(hg, p.Hkv - gi * hg);  // heads in this group (the last may be short)
+  x = r / (sz * Z);
+  const int r2 = r - x * (sz * Z);
+  kvh = gi * hg + r2 % sz;
+  z = r2 / sz;
 }
 
 // ------------------------------------------------------------------ varlen: tile prefix sums
