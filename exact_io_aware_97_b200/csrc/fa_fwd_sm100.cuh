@@ -9,8 +9,9 @@
 // and the per-row logsumexp are written to device memory.
 //
 // B200 mapping (one persistent CTA per SM, 384 threads):
-//   warps 0-3   softmax for query tile 0 (thread = row), then its epilogue
-//   warps 4-7   softmax for query tile 1
+//   warps 0-3   softmax for query tile 0 (thread = row), then its epilogue (O / l; bf16 O
+//               goes out through shared memory by TMA stores)
+//   warps 4-7   the same for query tile 1
 //   warp  8     tcgen05.mma issuer and TMEM owner
 //   warp  9     TMA producer
 //   warps 10-11 idle (they complete the control warpgroup for the register split)
