@@ -16,9 +16,11 @@
 //   warp  9     TMA producer
 //   warps 10-11 idle (they complete the control warpgroup for the register split)
 // The issuing warps run converged and let one elected lane issue each group of instructions.
-// A work unit is 256 query rows (two 128-row tiles) of one (sequence, query head).  Units
-// are ordered longest-first (causal cost grows with the query tile index) and dealt to
-// CTAs in a snake order.  K and V tiles (128 keys each) flow through a shared-memory ring
+// A work unit is two 128-row query tiles that share their K/V tiles: 256 rows of one
+// (sequence, query head), or (hpair) 128 rows of two query heads of one K/V group, which see
+// exactly the same keys, so no causal step runs with one tile.  Units are ordered
+// longest-first (causal cost grows with the query tile index) and dealt to CTAs in a snake
+// order.  K and V tiles (128 keys each) flow through a shared-memory ring
 // of full/empty mbarriers.  TMEM (512 columns): S0 | S1 (128 fp32 columns each, P is
 // written back over the first 64 columns of its S as packed bf16) | O0 | O1 (d columns).
 // The MMA order S0(j+1) after O0 += P0(j) V(j) and S1(j+1) after O1 += P1(j) V(j) lets the
@@ -48,11 +50,12 @@ struct FwdParams {
   float o_scale;  // multiplies O at the end (fp8: the v dequantisation factor; else 1)
   int T;          // fixed length: 256-row units per (sequence, head)
   int o_tma;      // bf16 O written through shared memory by TMA stores (tmO describes o)
+  int hpair;      // 1: a unit is 128 rows of two query heads of one K/V group (else 256 rows of one)
 };
 
 constexpr int kBM = 128;        // query rows per tile
 constexpr int kBN = 128;        // keys per K/V tile
-constexpr int kUnitRows = 256;  // two query tiles per work unit
+constexpr int kUnitRows = 256;  // two query tiles per work unit (128 rows x 2 heads with hpair)
 constexpr int kFwdThreads = 384;
 // Register split by warpgroup, set with setmaxnreg after the common prologue.  The launch
 // gives 384 threads x 168 registers = 64512; softmax warpgroups take 2 x 128 x 208 and the
@@ -107,7 +110,8 @@ struct FwdCfg {
 
 // Geometry of one work unit as every role sees it.
 struct Unit {
-  int b, h, kvh;
+  int b, h, kvh;         // h: query head of tile 0
+  int rstep, hstep;      // tile 1 = tile 0 moved by rstep rows and hstep heads
   int q_start, k_start;  // first row of the sequence in q/o and in k/v
   int nq, nk;
   int row0;   // first query row of the unit within the sequence
@@ -139,12 +143,14 @@ __device__ __forceinline__ int kv_tiles_for(int last_row, int nq, int nk, int ca
 __device__ __forceinline__ void decode_unit(const FwdParams& p, const SchedShared& s, UnitWalker& w, int u,
                                             Unit& out) {
   int b, t, h;
+  const int hp = p.hpair;
+  const int hunits = p.Hq >> hp;  // units per (sequence, level)
   if (p.cu == nullptr) {
-    const int per_level = p.B * p.Hq;
+    const int per_level = p.B * hunits;
     const int level = u / per_level;
     const int off = u - level * per_level;
-    b = off / p.Hq;
-    h = off - b * p.Hq;
+    b = off / hunits;
+    h = (off - b * hunits) << hp;
     t = s.T - 1 - level;
     out.q_start = b * p.Nq;
     out.k_start = b * p.Nk;
@@ -152,14 +158,14 @@ __device__ __forceinline__ void decode_unit(const FwdParams& p, const SchedShare
     out.nk = p.Nk;
   } else {
     for (;;) {
-      const int sz = s.cnt[s.T - 1 - w.level] * p.Hq;
+      const int sz = s.cnt[s.T - 1 - w.level] * hunits;
       if (u < w.level_start + sz) break;
       w.level_start += sz;
       ++w.level;
     }
     const int off = u - w.level_start;
-    const int r = off / p.Hq;
-    h = off - r * p.Hq;
+    const int r = off / hunits;
+    h = (off - r * hunits) << hp;
     b = s.sigma[r];
     t = s.T - 1 - w.level;
     const int c0 = __ldg(p.cu + b), c1 = __ldg(p.cu + b + 1);
@@ -171,9 +177,11 @@ __device__ __forceinline__ void decode_unit(const FwdParams& p, const SchedShare
   out.b = b;
   out.h = h;
   out.kvh = h / p.G;
-  out.row0 = t * kUnitRows;
+  out.row0 = t * (kUnitRows >> hp);
+  out.rstep = hp ? 0 : kBM;
+  out.hstep = hp;
   for (int i = 0; i < 2; ++i) {
-    const int r0 = out.row0 + i * kBM;
+    const int r0 = out.row0 + i * out.rstep;
     out.valid[i] = r0 < out.nq;
     out.n[i] = out.valid[i] ? kv_tiles_for(min(r0 + kBM - 1, out.nq - 1), out.nq, out.nk, p.causal) : 0;
   }
@@ -278,7 +286,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
   sch.cnt = cnt;
   if (p.cu == nullptr) {
     sch.T = p.T;
-    sch.U = p.T * p.B * p.Hq;
+    sch.U = p.T * p.B * (p.Hq >> p.hpair);
     __syncthreads();
   } else {
     __syncthreads();  // sched_misc initialised
@@ -290,7 +298,8 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       const int c0 = __ldg(p.cu + b), c1 = __ldg(p.cu + b + 1);
       bad |= (c1 < c0) | (b == 0 && c0 < 0) | (b == p.B - 1 && c1 > p.Nq);
       const int len = c1 - c0;
-      const int nt = len > 0 ? (len + kUnitRows - 1) / kUnitRows : 0;
+      const int ur = kUnitRows >> p.hpair;
+      const int nt = len > 0 ? (len + ur - 1) / ur : 0;
       atomicMax(&sched_misc[0], nt);
       atomicAdd(&sched_misc[1], nt);
     }
@@ -302,11 +311,12 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
     const int T = min(sched_misc[0], kMaxVarlenT);
     for (int b = threadIdx.x; b < p.B; b += blockDim.x) {
       const int lb = __ldg(p.cu + b + 1) - __ldg(p.cu + b);
-      const int nb = lb > 0 ? (lb + kUnitRows - 1) / kUnitRows : 0;
+      const int ur = kUnitRows >> p.hpair;
+      const int nb = lb > 0 ? (lb + ur - 1) / ur : 0;
       int rank = 0;
       for (int b2 = 0; b2 < p.B; ++b2) {
         const int l2 = __ldg(p.cu + b2 + 1) - __ldg(p.cu + b2);
-        const int n2 = l2 > 0 ? (l2 + kUnitRows - 1) / kUnitRows : 0;
+        const int n2 = l2 > 0 ? (l2 + ur - 1) / ur : 0;
         rank += (n2 > nb) || (n2 == nb && b2 < b);
       }
       sigma[rank] = (uint16_t)b;
@@ -315,14 +325,14 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       int c = 0;
       for (int b2 = 0; b2 < p.B; ++b2) {
         const int l2 = __ldg(p.cu + b2 + 1) - __ldg(p.cu + b2);
-        const int n2 = l2 > 0 ? (l2 + kUnitRows - 1) / kUnitRows : 0;
+        const int n2 = l2 > 0 ? (l2 + (kUnitRows >> p.hpair) - 1) / (kUnitRows >> p.hpair) : 0;
         c += n2 > t;
       }
       cnt[t] = c;
     }
     __syncthreads();
     sch.T = T;
-    sch.U = sched_misc[1] * p.Hq;
+    sch.U = sched_misc[1] * (p.Hq >> p.hpair);
   }
 
   tc_fence_before();
@@ -348,8 +358,8 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         mbar_arrive_expect_tx_elect(q_full, ntile * C::kTileBytes);
         for (int i = 0; i < ntile; ++i)
           for (int c = 0; c < C::kPanels; ++c)
-            tma_load_3d_elect(sQ + i * C::kTileBytes + c * C::kChunkBytes, &tmQ, c * C::kPanelCols, un.h,
-                        un.q_start + un.row0 + i * kBM, q_full);
+            tma_load_3d_elect(sQ + i * C::kTileBytes + c * C::kChunkBytes, &tmQ, c * C::kPanelCols,
+                              un.h + i * un.hstep, un.q_start + un.row0 + i * un.rstep, q_full);
         for (int j = 0; j < un.nmax && ok; ++j) {
           for (int kv = 0; kv < 2; ++kv) {
             const uint32_t slot = g % NS;
@@ -528,8 +538,9 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       const int my_valid = i ? un.valid[1] : un.valid[0];
       if (!my_valid) continue;
       const int n = i ? un.n[1] : un.n[0];
-      const int row = un.row0 + i * kBM + r;                       // row within the sequence
-      const int warp_row_min = un.row0 + i * kBM + (warp & 3) * 32;
+      const int row = un.row0 + i * un.rstep + r;                  // row within the sequence
+      const int warp_row_min = un.row0 + i * un.rstep + (warp & 3) * 32;
+      const int head = un.h + i * un.hstep;                        // query head of this tile
       const int diag = un.nk - un.nq;                              // causal offset
       float m_ref = -INFINITY, l = 0.f;
 
@@ -680,7 +691,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       pvcnt += n;
       const bool row_ok = row < un.nq;
       const float inv_l = l > 0.f ? p.o_scale / l : 0.f;
-      const size_t orow = ((size_t)(un.q_start + row) * p.Hq + un.h) * D;
+      const size_t orow = ((size_t)(un.q_start + row) * p.Hq + head) * D;
       // A warp whose 32 rows all lie in the sequence writes O by TMA: its rows go to a 1 KB
       // box of shared memory 16 columns at a time (two boxes in turn, the 32-byte swizzle
       // keeps the row-per-lane writes free of bank conflicts) and one lane stores each box.
@@ -727,7 +738,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
             fence_proxy_async_smem();
             __syncwarp();
             if (lane == 0) {
-              tma_store_3d(&tmO, box, 32 * c + e0, un.h, un.q_start + row);
+              tma_store_3d(&tmO, box, 32 * c + e0, head, un.q_start + row);
               bulk_commit_group();
             }
           }
@@ -754,8 +765,8 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       }
       if (row_ok && p.lse != nullptr) {
         const float v = l > 0.f ? (m_ref + log2f(l)) * kLn2 : -INFINITY;
-        const size_t li = (p.cu != nullptr) ? (size_t)un.h * p.Nq + un.q_start + row
-                                             : ((size_t)un.b * p.Hq + un.h) * p.Nq + row;
+        const size_t li = (p.cu != nullptr) ? (size_t)head * p.Nq + un.q_start + row
+                                             : ((size_t)un.b * p.Hq + head) * p.Nq + row;
         p.lse[li] = v;
       }
     }
