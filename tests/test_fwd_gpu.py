@@ -46,6 +46,11 @@ SMALL = [
     (1, 1000, 1000, 16, 2, 128, 1),
     (2, 384, 1500, 4, 4, 64, 0),
     (1, 200, 1029, 8, 1, 128, 1),  # Nq < Nk causal: bottom-right aligned window
+    # query-head pairs of one K/V group per unit (even group size): ragged last tile, three
+    # sequences; a single query row against a longer causal window; pairs that see no key
+    (3, 130, 130, 4, 2, 64, 1),
+    (2, 1, 300, 8, 2, 128, 1),
+    (1, 390, 260, 6, 3, 128, 1),   # G = 2: rows 0..129 of each head pair see no key
 ]
 
 
